@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""bench.py -- key-switches/s of CKKS hybrid key switching on B200.
+
+Default workload (one step = one key switch through pc_keyswitch):
+  N=2^16, L=24 ciphertext primes + alpha=4 special primes (31-bit), dnum=6,
+  one ciphertext at the top level (l=24), rotation key whose uniform half is
+  regenerated in-kernel from its ChaCha12 seed; inputs are seeded uniform
+  residues, rotated over enough (ciphertext, key) sets that the step's inputs
+  exceed the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--keys regen|stored] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+independent key switches (weak scaling, no data-path collective); the time is
+the max over ranks.  --impl reference times the plain CPU oracle on the host
+cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 2**20
+MODMUL_IMAD = 3      # IMAD-pipe instructions of one Shoup modular multiply
+IMAD_PER_SM_CLK = 64  # 32-bit IMAD lanes per SM per clock
+SMS = 148
+
+
+# ----------------------------------------------------------------- workloads
+
+def workload_counts(logN: int, L: int, alpha: int, l: int, regen: bool = True):
+    """Algorithmic work of one key switch at level l (spec v1 dataflow):
+    modular multiplies (butterflies, conversions, products), HBM bytes of the
+    inputs and outputs that must move, and ChaCha12 blocks."""
+    N = 1 << logN
+    beta = -(-l // alpha)
+    ll = l + alpha
+    half_logN = N // 2 * logN          # butterflies of one limb NTT
+    d = [min(alpha, l - j * alpha) for j in range(beta)]
+    intt_c1 = l * half_logN + l * N     # + one scale multiply per coefficient
+    modup_conv = sum(dj * (ll - dj) * N for dj in d)
+    modup_ntt = sum((ll - dj) for dj in d) * half_logN
+    inner = 2 * beta * ll * N
+    md_intt = 2 * alpha * half_logN + 2 * alpha * N
+    md_conv = 2 * alpha * l * N
+    md_ntt = 2 * l * half_logN
+    md_scale = 2 * l * N
+    modmuls = intt_c1 + modup_conv + modup_ntt + inner + md_intt + md_conv + md_ntt + md_scale
+    key_bytes = beta * ll * N * 4 * (1 if regen else 2)
+    bytes_ = 2 * l * N * 4 + key_bytes + 2 * l * N * 4
+    blocks = beta * ll * N // 8 if regen else 0
+    return {"modmuls": modmuls, "bytes": bytes_, "chacha_blocks": blocks}
+
+
+def stage_modmuls(logN: int, L: int, alpha: int, l: int):
+    """Modular multiplies done by each profiled stage (kernel) of one key switch."""
+    N = 1 << logN
+    logC = min(8, logN - 4)
+    logR = logN - logC
+    beta = -(-l // alpha)
+    ll = l + alpha
+    d = [min(alpha, l - j * alpha) for j in range(beta)]
+    ntarg = sum(ll - dj for dj in d)
+    return {
+        "intt_row_c1": l * (N // 2) * logC,
+        "intt_col_modup_scale": l * (N // 2) * logR + l * N,
+        "modup_bconv_col": sum(dj * (ll - dj) for dj in d) * N + ntarg * (N // 2) * logR,
+        "inner_chacha": ntarg * (N // 2) * logC + 2 * beta * ll * N + 2 * alpha * (N // 2) * logC,
+        "moddown_intt_col": 2 * alpha * (N // 2) * logR + 2 * alpha * N,
+        "moddown_bconv_col": 2 * alpha * l * N + 2 * l * (N // 2) * logR,
+        "moddown_finish": 2 * l * (N // 2) * logC + 2 * l * N,
+    }
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.device = device
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.device), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in open(self.path).read().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# --------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import datetime
+
+    from key_switching_b200 import pc, synth
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = synth.WORKLOADS[args.workload]
+    q, p = pc.chain(wl.logN, wl.bits, wl.L, wl.alpha)
+    ctx = pc.Context(wl.logN, q, p, device=local)
+    N, L, A = wl.N, wl.L, wl.alpha
+    regen = args.keys == "regen"
+    prim = q + p
+    stream = torch.cuda.current_stream()
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint32).view(np.int32)).cuda()
+
+    def make_key(seed_id):
+        b = np.stack([synth.uniform_residues(prim, N, seed_id, 0xB, j) for j in range(wl.dnum)])
+        a = None
+        if not regen:
+            a = dev(np.stack([synth.uniform_residues(prim, N, seed_id, 0xA, j) for j in range(wl.dnum)]))
+        return pc.KSK(synth.chacha_seed(seed_id, rank), dev(b), a)
+
+    launches_per_step = 7
+    if args.workload == "ntt_n16":
+        unit, metric = "limb-NTTs/s", "forward+inverse negacyclic NTT throughput at N=2^16 (1 B200)"
+        NPL = L + A
+        per_set = wl.n_ct * NPL * N * 4
+        nsets = max(2, math.ceil(2 * L2_BYTES / per_set))
+        sets = [dev(synth.uniform_residues_batch(prim, N, wl.n_ct, 40 + s, rank)) for s in range(nsets)]
+        units_per_step = 2 * wl.n_ct * NPL
+
+        def step(k):
+            x = sets[k % nsets]
+            ctx.ntt_fwd(x, 0, NPL, wl.n_ct, stream)
+            ctx.ntt_inv(x, 0, NPL, wl.n_ct, stream)
+        launches_per_step = 4
+        levels = [L]
+        work = None
+    else:
+        unit, metric = "key-switches/s", "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline"
+        if args.workload == "sweep_n17":
+            metric = "key-switches/s at N=2^17 level sweep 40..1 (1 B200)"
+        levels = list(wl.levels) if wl.levels else [L]
+        B = wl.n_ct
+        ctx.ensure_workspace(max(levels), B)
+        per_set = (B * (2 * L * N * 4) + B * wl.dnum * (L + A) * N * 4 * (1 if regen else 2))
+        nsets = max(2, math.ceil(2 * L2_BYTES / per_set)) if args.workload != "sweep_n17" else 1
+        sets = []
+        for s in range(nsets):
+            keys = [make_key(1000 * s + k + 1) for k in range(B)]
+            ct = dev(np.stack([np.stack([synth.uniform_residues(q, N, 50 + s, rank, k, h) for h in range(2)])
+                               for k in range(B)]))
+            sets.append((ct, keys))
+        out = torch.empty((B, 2, L, N), dtype=torch.int32, device="cuda")
+        units_per_step = B * len(levels)
+
+        def step(k):
+            ct, keys = sets[k % nsets]
+            for l in levels:
+                lN = l * N
+                if B == 1:
+                    # level-l ciphertext = the first l limbs of each half
+                    c0 = ct[0, 0, :l]
+                    c1 = ct[0, 1, :l]
+                    ctx.keyswitch(c0, c1, l, keys[0], out[0, 0, :l], out[0, 1, :l], stream)
+                else:
+                    ctx.keyswitch_batch(ct, B, l, keys, out, stream)
+        launches_per_step = 7 * len(levels)
+        work = [workload_counts(wl.logN, L, A, l, regen) for l in levels]
+
+    # warm-up, then exactly K timed steps between barriers
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    prof = args.workload != "ntt_n16"
+    if prof:
+        ctx.profile_begin(args.steps * len(levels))
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    stage_ms, ncalls = ctx.profile_end() if prof else ({}, 0)
+    if dist:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    total_units = units_per_step * args.steps * world
+    value = total_units / (ms * 1e-3)
+
+    res = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic (seeded uniform residues, "
+           "uniform key 'b' halves; ChaCha12 seeds)",
+           "config": {"workload": f"{wl.name}: N=2^{wl.logN}, L={L}, alpha={A}, dnum={wl.dnum}, "
+                      f"{wl.n_ct} ct/step, levels {levels[0]}..{levels[-1]}, key a-half "
+                      f"{'regenerated in-kernel (ChaCha12)' if regen else 'stored in HBM'}",
+                      "l2": f"inputs rotated over {nsets} sets of {per_set / 1e6:.1f} MB (> 126 MB L2)",
+                      "parallelism": f"replicas x{world}"},
+           "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+
+    if work is not None:
+        mm = sum(w["modmuls"] for w in work)
+        by = sum(w["bytes"] for w in work)
+        sec_per_step = ms * 1e-3 / args.steps / world * world  # per rank
+        sm_mhz = clk.get("sm_mhz") or 1965.0
+        peak_derived = SMS * IMAD_PER_SM_CLK * 1965e6 / MODMUL_IMAD
+        try:
+            peak_meas = pc.microbench(0, 2048, local) if rank == 0 else None
+        except Exception:
+            peak_meas = None
+        hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"] \
+            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 6650.0
+        t_roof = max(by / (hbm * 1e9), mm / peak_derived)
+        res["step_roofline"] = {"modmuls_per_step": mm * wl.n_ct, "hbm_bytes_per_step": by * wl.n_ct,
+                                "achieved_gbs": by * wl.n_ct / sec_per_step / 1e9,
+                                "achieved_tmodmul_s": mm * wl.n_ct / sec_per_step / 1e12,
+                                "t_roofline_us": t_roof * wl.n_ct * 1e6, "t_step_us": sec_per_step * 1e6,
+                                "frac": t_roof * wl.n_ct / sec_per_step,
+                                "modmul_peak_derived": peak_derived,
+                                "modmul_peak_microbench": peak_meas, "hbm_peak_gbs": hbm}
+        if stage_ms and ncalls:
+            smm = {}
+            for l in levels:
+                for kname, v in stage_modmuls(wl.logN, L, A, l).items():
+                    smm[kname] = smm.get(kname, 0) + v * wl.n_ct
+            tot = sum(stage_ms.values())
+            top = max(stage_ms, key=stage_ms.get)
+            per_launch_s = stage_ms[top] * 1e-3 / args.steps
+            ach = smm[top] / per_launch_s
+            res["roofline"] = {"bound": "alu", "kernel": top, "achieved": ach / 1e12,
+                               "peak": peak_derived / 1e12, "unit": "Tmodmul/s",
+                               "frac": ach / peak_derived, "traffic": None,
+                               "share": stage_ms[top] / tot if tot else None}
+            res["stage_ms_per_step"] = {k: v / args.steps for k, v in stage_ms.items()}
+
+    # end-to-end: host buffers through the same C-ABI call, copies timed
+    if not args.no_e2e and args.workload in ("rot1_n16", "relin_n12"):
+        ct0, keys0 = sets[0]
+        l = L
+        h_in = torch.empty((2, l, N), dtype=torch.int32).pin_memory()
+        h_in.copy_(ct0[0].cpu())
+        h_out = torch.empty((2, l, N), dtype=torch.int32).pin_memory()
+        d_in = torch.empty((2, l, N), dtype=torch.int32, device="cuda")
+        d_out = torch.empty((2, l, N), dtype=torch.int32, device="cuda")
+        ke = max(3, min(args.steps, 50))
+
+        def e2e_step():
+            d_in.copy_(h_in, non_blocking=True)
+            ctx.keyswitch(d_in[0], d_in[1], l, keys0[0], d_out[0], d_out[1], stream)
+            h_out.copy_(d_out, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        if dist:
+            t = torch.tensor([ems], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        res["e2e"] = {"value": ke * world / (ems * 1e-3), "unit": unit,
+                      "h2d_bytes_per_step": 2 * l * N * 4, "d2h_bytes_per_step": 2 * l * N * 4}
+
+    if rank == 0 and not args.no_cpu_baseline and args.workload in ("rot1_n16", "relin_n12"):
+        res["cpu_baseline"] = cpu_baseline(wl, q, p, budget_s=args.cpu_budget)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ------------------------------------------------------------ oracle timing
+
+def _oracle_inputs(wl, q, p):
+    import numpy as np
+    from key_switching_b200 import synth
+    from oracle import oracle as O
+    P = O.Params(wl.logN, q, p)
+    prim = [P.prime(g) for g in range(P.L + P.alpha)]
+    b = np.stack([synth.uniform_residues(prim, P.N, 1, 0xB, j) for j in range(P.dnum)])
+    l = wl.L
+    c0 = synth.uniform_residues(P.q[:l], P.N, 50, 0, 0, 0)
+    c1 = synth.uniform_residues(P.q[:l], P.N, 50, 0, 0, 1)
+    return O, P, b, c0, c1, l, synth.chacha_seed(1, 0)
+
+
+def cpu_baseline(wl, q, p, budget_s: float = 20.0):
+    """The oracle as it stands, single-threaded, on a bounded sample: as many
+    full key switches of the workload as fit in about budget_s seconds."""
+    O, P, b, c0, c1, l, seed = _oracle_inputs(wl, q, p)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        O.keyswitch(P, c0, c1, l, seed, b)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s or n >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "key-switches/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} full key switch(es) of {wl.name} (l={l}) in {dt:.1f} s, single thread"}
+
+
+def run_reference(args):
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return
+    from key_switching_b200 import pc, synth
+    wl = synth.WORKLOADS[args.workload]
+    q, p = pc.chain(wl.logN, wl.bits, wl.L, wl.alpha)
+    O, P, b, c0, c1, l, seed = _oracle_inputs(wl, q, p)
+    budget = args.cpu_budget * 6
+    t0 = time.perf_counter()
+    for _ in range(min(args.warmup, 1)):
+        O.keyswitch(P, c0, c1, l, seed, b)
+    t_one = max(1e-3, time.perf_counter() - t0)
+    steps = max(1, min(args.steps, int(budget / t_one)))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.keyswitch(P, c0, c1, l, seed, b)
+    dt = time.perf_counter() - t0
+    v = steps / dt
+    unit = "key-switches/s"
+    res = {"impl": "reference", "metric": "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline",
+           "value": v, "unit": unit, "n_gpus": 1, "steps": steps, "warmup": min(args.warmup, 1),
+           "ms_per_step": dt * 1e3 / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "u32", "data": "synthetic",
+           "config": {"workload": f"{wl.name}: N=2^{wl.logN}, L={wl.L}, alpha={wl.alpha}, dnum={wl.dnum}, "
+                      "1 ct/step at the top level, key a-half regenerated (ChaCha12)"},
+           "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle",
+                            "sample": f"{steps} of {args.steps} requested step(s), each one full key switch, "
+                                      "time-bounded, single thread"},
+           "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="rot1_n16",
+                    choices=["rot1_n16", "relin_n12", "batch16_n16", "ntt_n16", "sweep_n17"])
+    ap.add_argument("--keys", default="regen", choices=["regen", "stored"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

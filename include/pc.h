@@ -1,0 +1,203 @@
+/*
+ * pc.h -- C ABI of libpc: CKKS hybrid key switching over a 32-bit-word RNS
+ * basis on one NVIDIA B200 (sm_100a), with the uniform 'a' half of every
+ * key-switching key regenerated inside the kernel from a ChaCha12 seed.
+ *
+ * What the calls compute (the pages describe the operation, not its formula):
+ *   - Perseus README (github gladia-research-group/perseus), "Layout": the
+ *     device runtime provides the NTT and key switching over the 32-bit chain
+ *     (intro: kernels descend from a 32-bit GPU port of FIDESlib);
+ *   - same README, "What's inside": half of every key-switching key is
+ *     regenerated on the GPU from a ChaCha12 seed instead of being stored;
+ *   - "Perseus: A Full-Stack System for Homomorphic Model Inference"
+ *     (arxivlens summary), "Methodology": a ChaCha12 counter-mode expander.
+ * The formulas are the textbook ones (hybrid key switching of Han-Ki 2020;
+ * full-RNS CKKS of Cheon-Han-Kim-Kim-Song 2018 with the approximate FastBConv
+ * of Bajard-Eynard-Hasan-Zucca 2016), frozen as "spec v1" and stated at each
+ * call below.
+ *
+ * Conventions for every call:
+ *   - N = 2^logN, 10 <= logN <= 17.  Residues are uint32 in [0, q).
+ *   - Global prime index g: 0..L-1 are the ciphertext primes q_g, L..L+alpha-1
+ *     the special primes p_{g-L}.  At level l (1 <= l <= L, the number of q
+ *     limbs) the local limb t in [0, l+alpha) is q_t for t < l and p_{t-l}
+ *     otherwise.
+ *   - Digit j at level l: D_j = {q_{j*alpha} .. q_{min(j*alpha+alpha, l)-1}},
+ *     beta = ceil(l/alpha) digits (the last may be partial).
+ *   - Polynomials are limb-major: [limb][N] uint32, in the NTT domain
+ *     a_hat[k] = sum_n a[n] psi^((2 brv(k) + 1) n) mod q, psi the smallest
+ *     primitive 2N-th root of unity mod q, brv the logN-bit reversal.
+ *   - Pointers marked "device" are CUDA device pointers on the context's
+ *     device, 16-byte aligned (else PC_E_ALIGN).  The caller owns every data
+ *     buffer and the stream; no call allocates or frees device memory after
+ *     pc_ctx_create.  Calls are asynchronous on `stream` (a cudaStream_t, 0 =
+ *     legacy default stream); a return of PC_OK means "launched".
+ *   - Buffers must not overlap unless a call says so.
+ */
+#ifndef PC_H
+#define PC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define PC_OK 0
+#define PC_E_ARG (-1)       /* null pointer, level/size out of range, bad params */
+#define PC_E_ALIGN (-2)     /* a device pointer is not 16-byte aligned */
+#define PC_E_CUDA (-3)      /* a CUDA call or launch failed (see pc_strerror) */
+#define PC_E_DEVICE (-4)    /* a kernel reported an error through the device error word */
+#define PC_E_TIMEOUT (-5)   /* a bounded device wait gave up */
+#define PC_E_PRIME (-6)     /* a modulus is not prime, not = 1 mod 2N, or >= 2^31 */
+#define PC_E_WORKSPACE (-7) /* no workspace set, or smaller than pc_workspace_bytes */
+
+typedef struct pc_ctx pc_ctx; /* opaque; owns the device constant tables */
+typedef void *pc_stream;      /* a cudaStream_t */
+
+/* RNS basis.  q: host array of L ciphertext primes; p: host array of alpha
+ * special primes.  Every prime must be < 2^31 and = 1 mod 2N; all distinct.
+ * dnum must equal ceil(L/alpha). */
+typedef struct {
+    uint32_t logN, L, alpha, dnum;
+    const uint32_t *q;
+    const uint32_t *p;
+} pc_params;
+
+/* A key-switching key for s' -> s ("packed": seed + stored 'b' half).
+ *   seed: 32-byte ChaCha12 key of the 'a' half.
+ *   b:    device, [dnum][L+alpha][N], NTT domain, indexed by global prime:
+ *         b_{j,g} = -a_{j,g} s + e_j + [P]_{q_g} s' [q_g in D_j at the top level].
+ *   a:    device or NULL.  NULL: a_{j,g} is regenerated in-kernel (spec v1
+ *         mapping, see pc_expand_a).  Non-NULL: stored 'a' with b's layout. */
+typedef struct {
+    uint8_t seed[32];
+    const uint32_t *b;
+    const uint32_t *a;
+} pc_ksk;
+
+/* ---------------------------------------------------------------- */
+/* parameters and context                                            */
+/* ---------------------------------------------------------------- */
+
+/* NTT-friendly primes below 2^bits (bits <= 31), host only: scan
+ * k = floor((2^bits - 1)/2N) downward and keep c = k*2N + 1 when c is prime;
+ * writes the first `count` found (largest first).  Spec v1 assigns the first
+ * alpha of them to P and the next L to Q.  Returns PC_OK or PC_E_ARG. */
+int pc_gen_primes(uint32_t logN, uint32_t bits, uint32_t count, uint32_t *out);
+
+/* Validate the basis and build the device tables (twiddles, basis-conversion
+ * constants) on `device`.  On success *out owns them; this is the only call
+ * that allocates device memory.  Returns PC_OK, PC_E_ARG, PC_E_PRIME or
+ * PC_E_CUDA. */
+int pc_ctx_create(const pc_params *params, int device, pc_ctx **out);
+void pc_ctx_destroy(pc_ctx *ctx);
+
+/* psi (the smallest primitive 2N-th root) of global prime g, or 0 if g is out
+ * of range.  Host only. */
+uint32_t pc_psi(const pc_ctx *ctx, uint32_t g);
+
+/* Bytes of device scratch that pc_keyswitch / pc_keyswitch_batch (B
+ * ciphertexts), pc_modup and pc_moddown need at level l; and the call that
+ * hands such a buffer (device, 256-byte aligned, owned by the caller, kept
+ * until replaced) to the context.  Calls sharing one context and workspace
+ * must be ordered on one stream. */
+size_t pc_workspace_bytes(const pc_ctx *ctx, uint32_t l, uint32_t B);
+int pc_set_workspace(pc_ctx *ctx, void *dev, size_t bytes);
+
+/* ---------------------------------------------------------------- */
+/* operations                                                        */
+/* ---------------------------------------------------------------- */
+
+/* Negacyclic NTT, in place.  x: device, [batch][nlimbs][N]; limb k of every
+ * polynomial uses global prime first_prime + k (< L+alpha).  Forward maps
+ * coefficients to the NTT domain defined above; inverse is its exact inverse
+ * (N^-1 included).  Inputs in [0, q); outputs canonical. */
+int pc_ntt_fwd(pc_ctx *ctx, uint32_t *x, uint32_t first_prime, uint32_t nlimbs,
+               uint32_t batch, pc_stream stream);
+int pc_ntt_inv(pc_ctx *ctx, uint32_t *x, uint32_t first_prime, uint32_t nlimbs,
+               uint32_t batch, pc_stream stream);
+
+/* ModUp (spec v1: approximate fast basis conversion per digit).
+ * c1: device [l][N] NTT.  ext: device [beta][l+alpha][N] NTT, local limbs.
+ * With x_i = INTT(c1_i): y_i = x_i [Dhat_i^-1]_{q_i}, Dhat_i = prod of the
+ * digit's other primes; for t not in D_j, ext[j][t] = NTT_t(sum_i y_i [Dhat_i]_t
+ * mod t); for t in D_j, ext[j][t] = c1[t].  Needs the workspace. */
+int pc_modup(pc_ctx *ctx, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream stream);
+
+/* Key inner product with in-kernel ChaCha12 regeneration of 'a'.
+ * ext: device [beta][l+alpha][N] (pc_modup's output).  acc: device
+ * [2][l+alpha][N]; acc[0][t] = sum_j ext[j][t] b_{j,g(t)} mod t (b half),
+ * acc[1][t] = sum_j ext[j][t] a_{j,g(t)} mod t (a half).  a_{j,g} per
+ * pc_expand_a when k->a is NULL.  No workspace. */
+int pc_keyswitch_inner(pc_ctx *ctx, const uint32_t *ext, uint32_t l, const pc_ksk *k,
+                       uint32_t *acc, pc_stream stream);
+
+/* ModDown (spec v1: approximate conversion P -> Q_l, no rounding term).
+ * acc: device [2][l+alpha][N] NTT.  out: device [2][l][N] NTT with, for each
+ * half h, out[h][i] = (acc[h][i] - NTT(z_i)) [P^-1]_{q_i} where z_i =
+ * sum_p [INTT(acc[h][p]) Phat_p^-1]_p [Phat_p]_{q_i} mod q_i; i.e.
+ * floor(A/P) - v with v in [0, alpha).  Needs the workspace. */
+int pc_moddown(pc_ctx *ctx, const uint32_t *acc, uint32_t l, uint32_t *out, pc_stream stream);
+
+/* Full key switch s' -> s at level l: ModUp(c1), inner product, ModDown,
+ * c0' = c0 + out[0], c1' = out[1].  c0, c1, c0o, c1o: device [l][N] NTT.
+ * c0o may equal c0 and c1o may equal c1 (in place).  Needs the workspace. */
+int pc_keyswitch(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l,
+                 const pc_ksk *k, uint32_t *c0o, uint32_t *c1o, pc_stream stream);
+
+/* B independent key switches in one set of launches.  ct, out: device
+ * [B][2][l][N] (c0 then c1 of each ciphertext); keys: host array of B keys
+ * (ciphertext b uses keys[b]); out may equal ct.  1 <= B <= 64.  Needs the
+ * workspace for B ciphertexts. */
+int pc_keyswitch_batch(pc_ctx *ctx, const uint32_t *ct, uint32_t B, uint32_t l,
+                       const pc_ksk *keys, uint32_t *out, pc_stream stream);
+
+/* Test hook: write the regenerated 'a' words for level l.  a_out: device
+ * [beta][l+alpha][N], a_out[j][t][k] = a_{j,g(t)}[k] where (spec v1) block
+ * b = k/8 of ChaCha12 with state words (constants "expand 32-byte k", seed as
+ * eight little-endian words, counter b, g, j, 0x61) gives out[16], and
+ * a = (out[2(k%8)+1] * 2^32 + out[2(k%8)]) mod q_g. */
+int pc_expand_a(pc_ctx *ctx, const uint8_t seed[32], uint32_t l, uint32_t *a_out,
+                pc_stream stream);
+
+/* Synchronise the context's device and read its device error word; returns
+ * PC_OK, PC_E_DEVICE (and clears the word), or PC_E_CUDA. */
+int pc_check(pc_ctx *ctx);
+
+/* Human-readable text for a status code (the last CUDA error for PC_E_CUDA). */
+const char *pc_strerror(int code);
+
+/* ---------------------------------------------------------------- */
+/* measurement                                                       */
+/* ---------------------------------------------------------------- */
+
+/* Integer-throughput microbenchmark on `device`: runs `iters` rounds of
+ * independent modular-multiply chains (kind 0: Shoup multiply by a constant,
+ * the form the NTT and basis conversions use; kind 1: Montgomery multiply of
+ * two variables; kind 2: ChaCha12 blocks) over all SMs and writes the
+ * operations per second to *ops_per_s (modmuls/s, or ChaCha blocks/s).
+ * Synchronous.  Returns PC_OK, PC_E_ARG or PC_E_CUDA. */
+int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s);
+
+/* Per-kernel timing of pc_keyswitch / pc_keyswitch_batch, for measurement.
+ * pc_profile_begin creates CUDA events (host call, not on the hot path) for up
+ * to max_calls key-switch calls; each later call records one event before
+ * each of its PC_PROFILE_STAGES kernels and one after the last, on its stream.
+ * pc_profile_end synchronises, writes into ms[PC_PROFILE_STAGES] the summed
+ * milliseconds of each stage over the recorded calls (stages: 0 inverse row
+ * pass of c1, 1 inverse column pass + ModUp scale, 2 ModUp basis conversion +
+ * forward column pass, 3 inner product with ChaCha12 + special-limb inverse
+ * row pass, 4 special-limb inverse column pass, 5 ModDown basis conversion +
+ * forward column pass, 6 ModDown finish), sets *calls, and releases the
+ * events.  Returns PC_OK, PC_E_ARG or PC_E_CUDA. */
+#define PC_PROFILE_STAGES 7
+int pc_profile_begin(pc_ctx *ctx, uint32_t max_calls);
+int pc_profile_end(pc_ctx *ctx, float *ms, uint32_t *calls);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PC_H */

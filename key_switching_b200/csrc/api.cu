@@ -1,0 +1,608 @@
+// api.cu -- libpc host side: parameter checks, device constant tables, the
+// extern "C" entry points declared in include/pc.h, and argument marshalling
+// into the kernels of kernels.cu.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "pc_internal.h"
+
+using pc::u32;
+using pc::u64;
+
+namespace {
+
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda = e;
+    return PC_E_CUDA;
+}
+
+// ---------------------------------------------------------------- host math
+
+u32 mulm(u32 a, u32 b, u32 q) { return (u32)(((u64)a * b) % q); }
+
+u32 powm(u32 a, u64 e, u32 q) {
+    u64 r = 1, x = a % q;
+    for (; e; e >>= 1) {
+        if (e & 1) r = r * x % q;
+        x = x * x % q;
+    }
+    return (u32)(r % q);
+}
+
+u32 invm(u32 a, u32 q) { return powm(a, q - 2, q); }
+
+u32 shoup_of(u32 w, u32 q) { return (u32)(((u64)w << 32) / q); }
+
+// strong-probable-prime test to the bases 2, 3, 5, 7, 11: exact for every
+// n < 2,152,302,898,747 (Jaeschke 1993), so for all 32-bit n
+bool is_prime32(u32 n) {
+    if (n < 2) return false;
+    static const u32 small[] = {2, 3, 5, 7, 11, 13};
+    for (u32 p : small) {
+        if (n == p) return true;
+        if (n % p == 0) return false;
+    }
+    u32 d = n - 1;
+    int s = 0;
+    while (!(d & 1)) { d >>= 1; ++s; }
+    static const u32 bases[] = {2, 3, 5, 7, 11};
+    for (u32 a : bases) {
+        u32 x = powm(a, d, n);
+        if (x == 1 || x == n - 1) continue;
+        bool witness = true;
+        for (int i = 1; i < s && witness; ++i) {
+            x = mulm(x, x, n);
+            if (x == n - 1) witness = false;
+        }
+        if (witness) return false;
+    }
+    return true;
+}
+
+// The smallest primitive 2N-th root of unity mod q.  Find one root c (a
+// power x^((q-1)/2N) with c^N = -1), then every primitive 2N-th root is c^k
+// for odd k < 2N; take the minimum over them.
+u32 min_primitive_root_2n(u32 q, u32 logN) {
+    const u64 N = 1ull << logN, twoN = 2 * N;
+    if ((q - 1) % twoN) return 0;
+    u32 c = 0;
+    for (u32 x = 2; x < q && !c; ++x) {
+        u32 y = powm(x, (q - 1) / twoN, q);
+        if (powm(y, N, q) == q - 1) c = y;
+    }
+    if (!c) return 0;
+    const u32 c2 = mulm(c, c, q);
+    u32 best = c, r = c;
+    for (u64 k = 1; k < N; ++k) {
+        r = mulm(r, c2, q);
+        if (r < best) best = r;
+    }
+    return best;
+}
+
+u32 brv(u32 x, u32 bits) {
+    u32 r = 0;
+    for (u32 i = 0; i < bits; ++i) r |= ((x >> i) & 1u) << (bits - 1 - i);
+    return r;
+}
+
+// -u^-1 mod 2^32 for odd u (Newton iteration)
+u32 neg_inv32(u32 u) {
+    u32 x = u;  // correct to 3 bits
+    for (int i = 0; i < 5; ++i) x *= 2 - u * x;
+    return 0u - x;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+// workspace regions for B ciphertexts at level l (words)
+struct Layout {
+    size_t w1, t, acc, u, total;  // offsets and total, in words
+    size_t w1z, tz, accz, uz;     // per-ciphertext strides
+};
+Layout layout(const pc_ctx *c, u32 l, u32 B) {
+    Layout L{};
+    const size_t N = c->N, ll = l + c->alpha, beta = (l + c->alpha - 1) / c->alpha;
+    L.w1z = l * N;
+    L.tz = beta * ll * N;
+    L.accz = 2 * ll * N;
+    L.uz = 2 * (size_t)l * N;
+    L.w1 = 0;
+    L.t = L.w1 + B * L.w1z;
+    L.acc = L.t + B * L.tz;
+    L.u = L.acc + B * L.accz;
+    L.total = L.u + B * L.uz;
+    return L;
+}
+
+int check_ksk(const pc_ctx *c, const pc_ksk *k) {
+    if (!k || !k->b) return PC_E_ARG;
+    if (!aligned16(k->b) || (k->a && !aligned16(k->a))) return PC_E_ALIGN;
+    (void)c;
+    return PC_OK;
+}
+
+void seed_words(const uint8_t s[32], u32 out[8]) {
+    for (int w = 0; w < 8; ++w)
+        out[w] = (u32)s[4 * w] | ((u32)s[4 * w + 1] << 8) | ((u32)s[4 * w + 2] << 16) |
+                 ((u32)s[4 * w + 3] << 24);
+}
+
+void prof_release(pc_ctx *c) {
+    if (!c->prof_ev) return;
+    for (size_t i = 0; i < (size_t)c->prof_max * (PC_PROFILE_STAGES + 1); ++i) cudaEventDestroy(c->prof_ev[i]);
+    delete[] c->prof_ev;
+    c->prof_ev = nullptr;
+    c->prof_max = c->prof_used = 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pc_gen_primes(uint32_t logN, uint32_t bits, uint32_t count, uint32_t *out) {
+    if (!out || logN < 1 || logN > 30 || bits < 2 || bits > 31) return PC_E_ARG;
+    const u64 twoN = 2ull << logN;
+    u64 k = (((u64)1 << bits) - 1) / twoN;
+    u32 found = 0;
+    while (found < count) {
+        if (k == 0) return PC_E_ARG;
+        const u64 cand = k * twoN + 1;
+        if (is_prime32((u32)cand)) out[found++] = (u32)cand;
+        --k;
+    }
+    return PC_OK;
+}
+
+int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
+    if (!P || !out || !P->q || !P->p) return PC_E_ARG;
+    *out = nullptr;
+    if (P->logN < 10 || P->logN > 17) return PC_E_ARG;
+    if (P->L < 1 || P->L > (u32)pc::MAX_L || P->alpha < 1 || P->alpha > (u32)pc::MAX_ALPHA) return PC_E_ARG;
+    if (P->dnum != (P->L + P->alpha - 1) / P->alpha) return PC_E_ARG;
+    const u32 N = 1u << P->logN, NP = P->L + P->alpha;
+    std::vector<u32> pr(NP);
+    for (u32 i = 0; i < P->L; ++i) pr[i] = P->q[i];
+    for (u32 i = 0; i < P->alpha; ++i) pr[P->L + i] = P->p[i];
+    for (u32 i = 0; i < NP; ++i) {
+        if (pr[i] >= (1u << 31) || pr[i] < 3 || (pr[i] - 1) % (2 * N) || !is_prime32(pr[i])) return PC_E_PRIME;
+        for (u32 j = 0; j < i; ++j)
+            if (pr[j] == pr[i]) return PC_E_PRIME;
+    }
+    DeviceGuard dg(device);
+    if (!dg.ok) return cuda_fail(cudaGetLastError());
+
+    pc_ctx *c = new (std::nothrow) pc_ctx();
+    if (!c) return PC_E_ARG;
+    c->device = device;
+    c->logN = P->logN;
+    c->N = N;
+    c->L = P->L;
+    c->alpha = P->alpha;
+    c->dnum = P->dnum;
+    c->NP = NP;
+    for (u32 i = 0; i < NP; ++i) c->primes[i] = pr[i];
+    cudaError_t e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device);
+    if (e != cudaSuccess) { delete c; return cuda_fail(e); }
+
+    const u32 logC = (P->logN - 4 < 8) ? P->logN - 4 : 8, logR = P->logN - logC;
+    const u32 C = 1u << logC, R = 1u << logR;
+    const u32 L = P->L, A = P->alpha, D = P->dnum;
+
+    // host images of every table
+    std::vector<pc::PrimeK> pk(NP);
+    std::vector<uint2> colF((size_t)NP * R), colI((size_t)NP * R);
+    std::vector<uint2> rowF((size_t)NP * N), rowI((size_t)NP * N);
+    std::vector<uint2> upScale((size_t)A * L, make_uint2(0, 0));
+    std::vector<u32> upConv((size_t)D * A * NP * A, 0);
+    std::vector<uint2> downScale(A);
+    std::vector<u32> downConv((size_t)L * A);
+    std::vector<uint2> pInv(L);
+    std::vector<u32> pw(N), pwi(N);
+
+    for (u32 g = 0; g < NP; ++g) {
+        const u32 q = pr[g];
+        const u32 psi = min_primitive_root_2n(q, P->logN);
+        if (!psi) { delete c; return PC_E_PRIME; }
+        c->psi[g] = psi;
+        const u32 psii = invm(psi, q);
+        pw[0] = 1;
+        pwi[0] = 1;
+        for (u32 k = 1; k < N; ++k) {
+            pw[k] = mulm(pw[k - 1], psi, q);
+            pwi[k] = mulm(pwi[k - 1], psii, q);
+        }
+        auto rev = [&](const std::vector<u32> &t, u32 k) { return t[brv(k, P->logN)]; };
+        for (u32 k = 0; k < R; ++k) {
+            const u32 a = rev(pw, k), b = rev(pwi, k);
+            colF[(size_t)g * R + k] = make_uint2(a, shoup_of(a, q));
+            colI[(size_t)g * R + k] = make_uint2(b, shoup_of(b, q));
+        }
+        for (u32 r = 0; r < R; ++r) {
+            const size_t base = (size_t)g * N + (size_t)r * C;
+            rowF[base] = make_uint2(0, 0);
+            rowI[base] = make_uint2(0, 0);
+            for (u32 k = 1; k < C; ++k) {
+                u32 s = 0;
+                while ((2u << s) <= k) ++s;
+                const u32 idx = (R + r) * (1u << s) + (k - (1u << s));
+                const u32 a = rev(pw, idx), b = rev(pwi, idx);
+                rowF[base + k] = make_uint2(a, shoup_of(a, q));
+                rowI[base + k] = make_uint2(b, shoup_of(b, q));
+            }
+        }
+        pc::PrimeK &K = pk[g];
+        memset(&K, 0, sizeof(K));
+        K.q = q;
+        K.qn = neg_inv32(q);
+        K.q1s = (u32)((1ull << 32) / q);
+        K.r32 = (u32)((1ull << 32) % q);
+        K.r32s = shoup_of(K.r32, q);
+        K.r64 = mulm(K.r32, K.r32, q);
+        K.r64s = shoup_of(K.r64, q);
+        K.ninv = invm(N % q, q);
+        K.ninvs = shoup_of(K.ninv, q);
+    }
+    // ModUp: digit j of size d covers q_{j A} .. q_{j A + d - 1}
+    for (u32 j = 0; j < D; ++j) {
+        for (u32 d = 1; d <= A; ++d) {
+            const u32 lo = j * A;
+            if (lo + d > L) continue;
+            for (u32 k = 0; k < d; ++k) {
+                const u32 i = lo + k, qi = pr[i];
+                u32 dh = 1;
+                for (u32 m = 0; m < d; ++m)
+                    if (m != k) dh = mulm(dh, pr[lo + m] % qi, qi);
+                const u32 s = mulm(invm(N % qi, qi), invm(dh, qi), qi);
+                upScale[(size_t)(d - 1) * L + i] = make_uint2(s, shoup_of(s, qi));
+                for (u32 g = 0; g < NP; ++g) {
+                    const u32 t = pr[g];
+                    u32 dt = 1;
+                    for (u32 m = 0; m < d; ++m)
+                        if (m != k) dt = mulm(dt, pr[lo + m] % t, t);
+                    upConv[(((size_t)j * A + (d - 1)) * NP + g) * A + k] = mulm(dt, (u32)((1ull << 32) % t), t);
+                }
+            }
+        }
+    }
+    // ModDown
+    for (u32 k = 0; k < A; ++k) {
+        const u32 p = pr[L + k];
+        u32 ph = 1;
+        for (u32 m = 0; m < A; ++m)
+            if (m != k) ph = mulm(ph, pr[L + m] % p, p);
+        const u32 s = mulm(invm(N % p, p), invm(ph, p), p);
+        downScale[k] = make_uint2(s, shoup_of(s, p));
+    }
+    for (u32 i = 0; i < L; ++i) {
+        const u32 qi = pr[i];
+        u32 Pm = 1;
+        for (u32 k = 0; k < A; ++k) {
+            Pm = mulm(Pm, pr[L + k] % qi, qi);
+            u32 ph = 1;
+            for (u32 m = 0; m < A; ++m)
+                if (m != k) ph = mulm(ph, pr[L + m] % qi, qi);
+            downConv[(size_t)i * A + k] = mulm(ph, (u32)((1ull << 32) % qi), qi);
+        }
+        const u32 pi = invm(Pm, qi);
+        pInv[i] = make_uint2(pi, shoup_of(pi, qi));
+    }
+
+    // one device allocation, 256-byte aligned sub-buffers
+    struct Piece { const void *src; size_t bytes; size_t off; };
+    std::vector<Piece> pieces = {
+        {pk.data(), pk.size() * sizeof(pc::PrimeK), 0},
+        {colF.data(), colF.size() * sizeof(uint2), 0},
+        {colI.data(), colI.size() * sizeof(uint2), 0},
+        {rowF.data(), rowF.size() * sizeof(uint2), 0},
+        {rowI.data(), rowI.size() * sizeof(uint2), 0},
+        {upScale.data(), upScale.size() * sizeof(uint2), 0},
+        {upConv.data(), upConv.size() * sizeof(u32), 0},
+        {downScale.data(), downScale.size() * sizeof(uint2), 0},
+        {downConv.data(), downConv.size() * sizeof(u32), 0},
+        {pInv.data(), pInv.size() * sizeof(uint2), 0},
+        {nullptr, 256, 0},  // device error word
+    };
+    size_t total = 0;
+    for (auto &p : pieces) {
+        p.off = total;
+        total += (p.bytes + 255) & ~(size_t)255;
+    }
+    void *blk = nullptr;
+    e = cudaMalloc(&blk, total);
+    if (e != cudaSuccess) { delete c; return cuda_fail(e); }
+    for (auto &p : pieces) {
+        if (p.src) e = cudaMemcpy((char *)blk + p.off, p.src, p.bytes, cudaMemcpyHostToDevice);
+        else e = cudaMemset((char *)blk + p.off, 0, p.bytes);
+        if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
+    }
+    auto at = [&](int i) { return (char *)blk + pieces[i].off; };
+    c->dev_block = blk;
+    c->dev_bytes = total;
+    pc::Tables &T = c->tab;
+    T.pk = (const pc::PrimeK *)at(0);
+    T.colF = (const uint2 *)at(1);
+    T.colI = (const uint2 *)at(2);
+    T.rowF = (const uint2 *)at(3);
+    T.rowI = (const uint2 *)at(4);
+    T.upScale = (const uint2 *)at(5);
+    T.upConv = (const u32 *)at(6);
+    T.downScale = (const uint2 *)at(7);
+    T.downConv = (const u32 *)at(8);
+    T.pInv = (const uint2 *)at(9);
+    T.err = (int *)at(10);
+    T.L = L;
+    T.alpha = A;
+    T.dnum = D;
+    T.NP = NP;
+    e = pc::prepare_kernels(c);
+    if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
+    *out = c;
+    return PC_OK;
+}
+
+void pc_ctx_destroy(pc_ctx *c) {
+    if (!c) return;
+    DeviceGuard dg(c->device);
+    prof_release(c);
+    if (c->dev_block) cudaFree(c->dev_block);
+    delete c;
+}
+
+uint32_t pc_psi(const pc_ctx *c, uint32_t g) { return (c && g < c->NP) ? c->psi[g] : 0; }
+
+size_t pc_workspace_bytes(const pc_ctx *c, uint32_t l, uint32_t B) {
+    if (!c || l < 1 || l > c->L || B < 1) return 0;
+    return layout(c, l, B).total * sizeof(u32);
+}
+
+int pc_set_workspace(pc_ctx *c, void *dev, size_t bytes) {
+    if (!c) return PC_E_ARG;
+    if (dev && ((uintptr_t)dev & 255u)) return PC_E_ALIGN;
+    c->ws = dev;
+    c->ws_bytes = dev ? bytes : 0;
+    return PC_OK;
+}
+
+int pc_ntt_fwd(pc_ctx *c, uint32_t *x, uint32_t first_prime, uint32_t nlimbs, uint32_t batch,
+               pc_stream stream) {
+    if (!c || !x || nlimbs < 1 || batch < 1 || first_prime + nlimbs > c->NP || batch > 65535) return PC_E_ARG;
+    if (!aligned16(x)) return PC_E_ALIGN;
+    DeviceGuard dg(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t z = (size_t)nlimbs * c->N;
+    cudaError_t e = pc::launch_col(c, true, x, x, first_prime, nlimbs, batch, z, z, 0, 0, s);
+    if (e == cudaSuccess) e = pc::launch_row(c, true, x, x, first_prime, nlimbs, batch, z, z, true, s);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+int pc_ntt_inv(pc_ctx *c, uint32_t *x, uint32_t first_prime, uint32_t nlimbs, uint32_t batch,
+               pc_stream stream) {
+    if (!c || !x || nlimbs < 1 || batch < 1 || first_prime + nlimbs > c->NP || batch > 65535) return PC_E_ARG;
+    if (!aligned16(x)) return PC_E_ALIGN;
+    DeviceGuard dg(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t z = (size_t)nlimbs * c->N;
+    cudaError_t e = pc::launch_row(c, false, x, x, first_prime, nlimbs, batch, z, z, false, s);
+    if (e == cudaSuccess) e = pc::launch_col(c, false, x, x, first_prime, nlimbs, batch, z, z, 1, 0, s);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+static int need_ws(const pc_ctx *c, u32 l, u32 B) {
+    if (!c->ws || c->ws_bytes < layout(c, l, B).total * sizeof(u32)) return PC_E_WORKSPACE;
+    return PC_OK;
+}
+
+int pc_modup(pc_ctx *c, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream stream) {
+    if (!c || !c1 || !ext || l < 1 || l > c->L) return PC_E_ARG;
+    if (!aligned16(c1) || !aligned16(ext)) return PC_E_ALIGN;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const Layout Lw = layout(c, l, 1);
+    u32 *w1 = (u32 *)c->ws + Lw.w1;
+    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, s);
+    if (e == cudaSuccess) e = pc::launch_col(c, false, w1, w1, 0, l, 1, 0, 0, 2, l, s);
+    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 0, w1, 0, ext, 0, l, 1, s);
+    if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+int pc_keyswitch_inner(pc_ctx *c, const uint32_t *ext, uint32_t l, const pc_ksk *k, uint32_t *acc,
+                       pc_stream stream) {
+    if (!c || !ext || !acc || l < 1 || l > c->L) return PC_E_ARG;
+    if (int r = check_ksk(c, k)) return r;
+    if (!aligned16(ext) || !aligned16(acc)) return PC_E_ALIGN;
+    DeviceGuard dg(c->device);
+    pc::KeyPack kp{};
+    kp.b[0] = k->b;
+    kp.a[0] = k->a;
+    seed_words(k->seed, kp.seed[0]);
+    cudaError_t e = pc::launch_inner(c, false, ext, 0, nullptr, 0, acc, 0, l, kp, 1, k->a == nullptr, false,
+                                     (cudaStream_t)stream);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_stream stream) {
+    if (!c || !acc || !out || l < 1 || l > c->L) return PC_E_ARG;
+    if (!aligned16(acc) || !aligned16(out)) return PC_E_ALIGN;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const Layout Lw = layout(c, l, 1);
+    u32 *wacc = (u32 *)c->ws + Lw.acc, *wu = (u32 *)c->ws + Lw.u;
+    const size_t N = c->N, ll = l + c->alpha;
+    // special-prime limbs of both halves: inverse row pass into the workspace
+    cudaError_t e = pc::launch_row(c, false, acc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, false, s);
+    if (e == cudaSuccess) e = pc::launch_col(c, false, wacc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, 3, l, s);
+    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 1, wacc, 2 * ll * N, wu, 2 * l * N, l, 1, s);
+    if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, 0, acc, 0, nullptr, 0, out, out + l * N, 0, l, 1, s);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+// shared body of pc_keyswitch and pc_keyswitch_batch: B ciphertexts whose
+// c0 / c1 / outputs sit at stride `cz` words.
+static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u32 l, const pc_ksk *keys,
+                          u32 B, u32 *o0, u32 *o1, cudaStream_t s) {
+    const Layout Lw = layout(c, l, B);
+    u32 *ws = (u32 *)c->ws;
+    u32 *w1 = ws + Lw.w1, *wt = ws + Lw.t, *wacc = ws + Lw.acc, *wu = ws + Lw.u;
+    const size_t N = c->N, ll = l + c->alpha;
+    const bool regen = keys[0].a == nullptr;
+    for (u32 b = 1; b < B; ++b)
+        if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
+    // optional per-stage events (measurement only)
+    cudaEvent_t *ev = nullptr;
+    if (c->prof_ev && c->prof_used < c->prof_max) ev = c->prof_ev + (size_t)(c->prof_used++) * (PC_PROFILE_STAGES + 1);
+    auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
+    mark(0);
+    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, B, cz, Lw.w1z, false, s);
+    mark(1);
+    if (e == cudaSuccess) e = pc::launch_col(c, false, w1, w1, 0, l, B, Lw.w1z, Lw.w1z, 2, l, s);
+    mark(2);
+    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 0, w1, Lw.w1z, wt, Lw.tz, l, B, s);
+    mark(3);
+    for (u32 b0 = 0; e == cudaSuccess && b0 < B; b0 += pc::KEYS_PER_LAUNCH) {
+        const u32 nb = (B - b0 < (u32)pc::KEYS_PER_LAUNCH) ? B - b0 : (u32)pc::KEYS_PER_LAUNCH;
+        pc::KeyPack kp{};
+        for (u32 i = 0; i < nb; ++i) {
+            kp.b[i] = keys[b0 + i].b;
+            kp.a[i] = keys[b0 + i].a;
+            seed_words(keys[b0 + i].seed, kp.seed[i]);
+        }
+        e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, c1 + b0 * cz, cz, wacc + b0 * Lw.accz, Lw.accz, l, kp,
+                             nb, regen, true, s);
+    }
+    mark(4);
+    if (e == cudaSuccess)
+        e = pc::launch_col(c, false, wacc + l * N, wacc + l * N, c->L, c->alpha, 2 * B, ll * N, ll * N, 3, l, s);
+    mark(5);
+    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, s);
+    mark(6);
+    if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, c0, cz, o0, o1, cz, l, B, s);
+    mark(7);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+int pc_keyswitch(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
+                 uint32_t *c0o, uint32_t *c1o, pc_stream stream) {
+    if (!c || !c0 || !c1 || !c0o || !c1o || l < 1 || l > c->L) return PC_E_ARG;
+    if (int r = check_ksk(c, k)) return r;
+    if (!aligned16(c0) || !aligned16(c1) || !aligned16(c0o) || !aligned16(c1o)) return PC_E_ALIGN;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    return keyswitch_core(c, c0, c1, 0, l, k, 1, c0o, c1o, (cudaStream_t)stream);
+}
+
+int pc_keyswitch_batch(pc_ctx *c, const uint32_t *ct, uint32_t B, uint32_t l, const pc_ksk *keys,
+                       uint32_t *out, pc_stream stream) {
+    if (!c || !ct || !out || !keys || B < 1 || B > 64 || l < 1 || l > c->L) return PC_E_ARG;
+    for (u32 b = 0; b < B; ++b)
+        if (int r = check_ksk(c, &keys[b])) return r;
+    if (!aligned16(ct) || !aligned16(out)) return PC_E_ALIGN;
+    if (int r = need_ws(c, l, B)) return r;
+    DeviceGuard dg(c->device);
+    const size_t lN = (size_t)l * c->N;
+    return keyswitch_core(c, ct, ct + lN, 2 * lN, l, keys, B, out, out + lN, (cudaStream_t)stream);
+}
+
+int pc_expand_a(pc_ctx *c, const uint8_t seed[32], uint32_t l, uint32_t *a_out, pc_stream stream) {
+    if (!c || !seed || !a_out || l < 1 || l > c->L) return PC_E_ARG;
+    if (!aligned16(a_out)) return PC_E_ALIGN;
+    DeviceGuard dg(c->device);
+    u32 sw[8];
+    seed_words(seed, sw);
+    cudaError_t e = pc::launch_expand(c, sw, l, a_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+int pc_profile_begin(pc_ctx *c, uint32_t max_calls) {
+    if (!c || max_calls < 1 || max_calls > 100000) return PC_E_ARG;
+    DeviceGuard dg(c->device);
+    prof_release(c);
+    const size_t n = (size_t)max_calls * (PC_PROFILE_STAGES + 1);
+    c->prof_ev = new (std::nothrow) cudaEvent_t[n];
+    if (!c->prof_ev) return PC_E_ARG;
+    for (size_t i = 0; i < n; ++i) {
+        cudaError_t e = cudaEventCreate(&c->prof_ev[i]);
+        if (e != cudaSuccess) {
+            for (size_t k = 0; k < i; ++k) cudaEventDestroy(c->prof_ev[k]);
+            delete[] c->prof_ev;
+            c->prof_ev = nullptr;
+            return cuda_fail(e);
+        }
+    }
+    c->prof_max = max_calls;
+    c->prof_used = 0;
+    return PC_OK;
+}
+
+int pc_profile_end(pc_ctx *c, float *ms, uint32_t *calls) {
+    if (!c || !ms) return PC_E_ARG;
+    DeviceGuard dg(c->device);
+    for (int k = 0; k < PC_PROFILE_STAGES; ++k) ms[k] = 0.f;
+    if (calls) *calls = c->prof_used;
+    int rc = PC_OK;
+    for (uint32_t i = 0; i < c->prof_used && rc == PC_OK; ++i) {
+        cudaEvent_t *ev = c->prof_ev + (size_t)i * (PC_PROFILE_STAGES + 1);
+        cudaError_t e = cudaEventSynchronize(ev[PC_PROFILE_STAGES]);
+        for (int k = 0; k < PC_PROFILE_STAGES && e == cudaSuccess; ++k) {
+            float t = 0.f;
+            e = cudaEventElapsedTime(&t, ev[k], ev[k + 1]);
+            ms[k] += t;
+        }
+        if (e != cudaSuccess) rc = cuda_fail(e);
+    }
+    prof_release(c);
+    return rc;
+}
+
+int pc_check(pc_ctx *c) {
+    if (!c) return PC_E_ARG;
+    DeviceGuard dg(c->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    int word = 0;
+    e = cudaMemcpy(&word, c->tab.err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word) {
+        cudaMemset(c->tab.err, 0, sizeof(int));
+        return PC_E_DEVICE;
+    }
+    return PC_OK;
+}
+
+const char *pc_strerror(int code) {
+    switch (code) {
+        case PC_OK: return "ok";
+        case PC_E_ARG: return "invalid argument (null pointer, level or size out of range, bad parameters)";
+        case PC_E_ALIGN: return "device pointer not 16-byte aligned (workspace: 256-byte)";
+        case PC_E_CUDA: return cudaGetErrorString(g_last_cuda);
+        case PC_E_DEVICE: return "a kernel reported an error through the device error word";
+        case PC_E_TIMEOUT: return "a bounded device wait gave up";
+        case PC_E_PRIME: return "modulus not prime, not 1 mod 2N, repeated, or >= 2^31";
+        case PC_E_WORKSPACE: return "workspace missing or smaller than pc_workspace_bytes";
+        default: return "unknown status code";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// chacha.cuh -- ChaCha12 block function in registers (Bernstein 2008).
+//
+// Used to regenerate the uniform 'a' half of a key-switching key inside the
+// inner-product kernel instead of reading it from HBM (Perseus README, "What's
+// inside": in-kernel key regeneration from a ChaCha12 seed; arxivlens summary
+// of the Perseus paper, "Methodology": ChaCha12 counter-mode expander).
+//
+// Spec v1 state: words 0..3 "expand 32-byte k", 4..11 the 32-byte seed as
+// little-endian words, 12 the block counter, 13 the global prime index,
+// 14 the digit, 15 the tag 0x61.  Six double rounds, then the input state is
+// added word-wise.
+#pragma once
+#include <cstdint>
+
+namespace pc {
+
+__device__ __forceinline__ uint32_t rotl32(uint32_t x, int r) { return __funnelshift_l(x, x, r); }
+
+#define PC_QR(a, b, c, d)                  \
+    a += b; d ^= a; d = rotl32(d, 16);     \
+    c += d; b ^= c; b = rotl32(b, 12);     \
+    a += b; d ^= a; d = rotl32(d, 8);      \
+    c += d; b ^= c; b = rotl32(b, 7);
+
+// out[16] = ChaCha12(seed words k[8], counter, g, j)
+__device__ __forceinline__ void chacha12_block(const uint32_t k[8], uint32_t ctr, uint32_t g,
+                                               uint32_t j, uint32_t out[16]) {
+    const uint32_t c0 = 0x61707865u, c1 = 0x3320646eu, c2 = 0x79622d32u, c3 = 0x6b206574u;
+    uint32_t x0 = c0, x1 = c1, x2 = c2, x3 = c3;
+    uint32_t x4 = k[0], x5 = k[1], x6 = k[2], x7 = k[3];
+    uint32_t x8 = k[4], x9 = k[5], x10 = k[6], x11 = k[7];
+    uint32_t x12 = ctr, x13 = g, x14 = j, x15 = 0x61u;
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+        PC_QR(x0, x4, x8, x12);
+        PC_QR(x1, x5, x9, x13);
+        PC_QR(x2, x6, x10, x14);
+        PC_QR(x3, x7, x11, x15);
+        PC_QR(x0, x5, x10, x15);
+        PC_QR(x1, x6, x11, x12);
+        PC_QR(x2, x7, x8, x13);
+        PC_QR(x3, x4, x9, x14);
+    }
+    out[0] = x0 + c0; out[1] = x1 + c1; out[2] = x2 + c2; out[3] = x3 + c3;
+    out[4] = x4 + k[0]; out[5] = x5 + k[1]; out[6] = x6 + k[2]; out[7] = x7 + k[3];
+    out[8] = x8 + k[4]; out[9] = x9 + k[5]; out[10] = x10 + k[6]; out[11] = x11 + k[7];
+    out[12] = x12 + ctr; out[13] = x13 + g; out[14] = x14 + j; out[15] = x15 + 0x61u;
+}
+#undef PC_QR
+
+}  // namespace pc

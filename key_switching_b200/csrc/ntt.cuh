@@ -1,0 +1,174 @@
+// ntt.cuh -- negacyclic NTT building blocks for sm_100a.
+//
+// Transform (spec v1; Longa-Naehrig merged-psi Cooley-Tukey network):
+//   a_hat[k] = sum_n a[n] psi^((2 brv(k) + 1) n) mod q, bit-reversed order.
+// Stage s (0-based) pairs elements at distance N >> (s+1); the butterfly whose
+// lower element is X uses psi_rev[(1 << s) + (X >> (logN - s))], with
+// psi_rev[k] = psi^brv(k).  The inverse runs the stages backwards with
+// Gentleman-Sande butterflies and psi^-1 powers, then scales by N^-1.
+//
+// B200 decomposition: N = R x C viewed as R rows of C contiguous words.
+//   - stages 0..logR-1 only pair elements of the same column: the "column
+//     pass", R-point transforms on C columns, every column using the same
+//     twiddles psi_rev[1..R-1];
+//   - stages logR..logN-1 stay inside a row: the "row pass", C-point
+//     transforms whose row-r twiddle for local stage s and group i is
+//     psi_rev[(R + r) 2^s + i]; they are re-laid out per row as
+//     RT[r][(1 << s) + i] so one row's table is C contiguous entries.
+// Every pass is a "line transform" of length M = 2^m (M = R or C): each
+// thread keeps 16 elements in registers and runs up to four stages (one
+// radix-16 phase) on them; phases exchange through shared memory.  A line
+// of M elements is handled by M/16 threads.
+#pragma once
+#include "modarith.cuh"
+
+namespace pc {
+
+// One phase: stages [S0, S0+K) of a length-2^LOGM line transform.
+// Register r = g*2^K + m holds element x_of(lt, r) of the thread's line.
+template <int LOGM, int S0, int K>
+struct Phase {
+    static constexpr int M = 1 << LOGM;
+    static constexpr int LOGD = LOGM - S0 - K;  // smallest distance of the phase
+    static constexpr int D = 1 << LOGD;
+    static constexpr int KK = 1 << K;  // members per group
+    static constexpr int G = 16 / KK;  // groups per thread
+    static constexpr int T = M / 16;   // threads per line
+    static_assert(K >= 1 && K <= 4 && LOGD >= 0, "bad phase");
+
+    __device__ static __forceinline__ int pair(int lt, int g) { return lt + g * T; }
+    __device__ static __forceinline__ int x_of(int lt, int r) {
+        const int g = r / KK, m = r % KK;
+        const int p = pair(lt, g);
+        return ((p >> LOGD) << (LOGD + K)) + (m << LOGD) + (p & (D - 1));
+    }
+
+    // forward stages; tw(idx) returns {w, w'} for table index idx in [1, M)
+    template <class TW>
+    __device__ static __forceinline__ void fwd(u32 v[16], int lt, const TW &tw, u32 q) {
+#pragma unroll
+        for (int u = 0; u < K; ++u) {
+            const int h = KK >> (u + 1);  // member distance at this sub-stage
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const int hi = pair(lt, g) >> LOGD;
+#pragma unroll
+                for (int b = 0; b < (1 << u); ++b) {
+                    const uint2 w = tw((1 << (S0 + u)) + (hi << u) + b);
+#pragma unroll
+                    for (int a = b * (KK >> u); a < b * (KK >> u) + h; ++a)
+                        bf_ct(v[g * KK + a], v[g * KK + a + h], w.x, w.y, q);
+                }
+            }
+        }
+    }
+
+    template <class TW>
+    __device__ static __forceinline__ void inv(u32 v[16], int lt, const TW &tw, u32 q) {
+#pragma unroll
+        for (int u = K - 1; u >= 0; --u) {
+            const int h = KK >> (u + 1);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const int hi = pair(lt, g) >> LOGD;
+#pragma unroll
+                for (int b = 0; b < (1 << u); ++b) {
+                    const uint2 w = tw((1 << (S0 + u)) + (hi << u) + b);
+#pragma unroll
+                    for (int a = b * (KK >> u); a < b * (KK >> u) + h; ++a)
+                        bf_gs(v[g * KK + a], v[g * KK + a + h], w.x, w.y, q);
+                }
+            }
+        }
+    }
+};
+
+// Phase partition of a length-2^LOGM line: [0,4), [4,8), [8,LOGM).
+template <int LOGM>
+struct Plan {
+    static_assert(LOGM >= 4 && LOGM <= 9, "line length 16..512");
+    static constexpr int NPH = LOGM <= 4 ? 1 : (LOGM <= 8 ? 2 : 3);
+    using P0 = Phase<LOGM, 0, (LOGM < 4 ? LOGM : 4)>;
+    using P1 = Phase<LOGM, 4, (LOGM > 4 ? (LOGM - 4 < 4 ? LOGM - 4 : 4) : 1)>;
+    using P2 = Phase<LOGM, 8, (LOGM > 8 ? LOGM - 8 : 1)>;
+    // element held by register r at the start / end of a forward transform
+    __device__ static __forceinline__ int fwd_in(int lt, int r) { return P0::x_of(lt, r); }
+    __device__ static __forceinline__ int fwd_out(int lt, int r) {
+        if constexpr (NPH == 1) return P0::x_of(lt, r);
+        else if constexpr (NPH == 2) return P1::x_of(lt, r);
+        else return P2::x_of(lt, r);
+    }
+    // the inverse starts where the forward ends and ends where it starts
+    __device__ static __forceinline__ int inv_in(int lt, int r) { return fwd_out(lt, r); }
+    __device__ static __forceinline__ int inv_out(int lt, int r) { return fwd_in(lt, r); }
+};
+
+// Exchange the registers of phase A's layout into phase B's layout through
+// shared memory.  ADDR(x) gives the word address of element x of the line.
+template <class PA, class PB, class ADDR>
+__device__ __forceinline__ void exchange(u32 v[16], u32 *sm, int lt, const ADDR &addr) {
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 16; ++r) sm[addr(PA::x_of(lt, r))] = v[r];
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 16; ++r) v[r] = sm[addr(PB::x_of(lt, r))];
+}
+
+// Full forward line transform: registers enter at Plan::fwd_in positions and
+// leave at Plan::fwd_out positions (lazy values in [0, 2q)).
+template <int LOGM, class ADDR, class TW>
+__device__ __forceinline__ void line_fwd(u32 v[16], u32 *sm, int lt, const ADDR &addr,
+                                         const TW &tw, u32 q) {
+    using PL = Plan<LOGM>;
+    PL::P0::fwd(v, lt, tw, q);
+    if constexpr (PL::NPH >= 2) {
+        exchange<typename PL::P0, typename PL::P1>(v, sm, lt, addr);
+        PL::P1::fwd(v, lt, tw, q);
+    }
+    if constexpr (PL::NPH >= 3) {
+        exchange<typename PL::P1, typename PL::P2>(v, sm, lt, addr);
+        PL::P2::fwd(v, lt, tw, q);
+    }
+}
+
+// Full inverse line transform (no N^-1): registers enter at Plan::inv_in
+// and leave at Plan::inv_out positions.
+template <int LOGM, class ADDR, class TW>
+__device__ __forceinline__ void line_inv(u32 v[16], u32 *sm, int lt, const ADDR &addr,
+                                         const TW &tw, u32 q) {
+    using PL = Plan<LOGM>;
+    if constexpr (PL::NPH >= 3) {
+        PL::P2::inv(v, lt, tw, q);
+        exchange<typename PL::P2, typename PL::P1>(v, sm, lt, addr);
+    }
+    if constexpr (PL::NPH >= 2) {
+        PL::P1::inv(v, lt, tw, q);
+        exchange<typename PL::P1, typename PL::P0>(v, sm, lt, addr);
+    }
+    PL::P0::inv(v, lt, tw, q);
+}
+
+// Geometry of a ring of degree 2^LOGN_: C = 2^LOGC-word rows, R = 2^LOGR rows.
+template <int LOGN_>
+struct Geo {
+    static constexpr int LOGN = LOGN_;
+    static constexpr int LOGC = (LOGN - 4 < 8) ? LOGN - 4 : 8;
+    static constexpr int LOGR = LOGN - LOGC;
+    static constexpr int N = 1 << LOGN, C = 1 << LOGC, R = 1 << LOGR;
+    // row pass: NL rows per CTA, C/16 threads per row
+    static constexpr int TPR = C / 16;
+    static constexpr int NL = (4096 / C < R) ? 4096 / C : R;
+    static constexpr int ROW_THREADS = NL * TPR;
+    static constexpr int ROW_BLOCKS = R / NL;
+    static constexpr int ROW_LS = C + C / 16;  // padded row stride in shared memory
+    // column pass: W columns per CTA, R/16 threads per column
+    static constexpr int TPCOL = R / 16;
+    static constexpr int W = (4096 / R < C) ? 4096 / R : C;
+    static constexpr int COL_THREADS = W * TPCOL;
+    static constexpr int COL_BLOCKS = C / W;
+    static constexpr int COL_LS = W + 1;  // padded shared-memory row stride of a column tile
+    static_assert(LOGC >= 4 && LOGR >= 4 && LOGR <= 9, "supported 2^8..2^17 (R,C >= 16)");
+};
+
+}  // namespace pc

@@ -1,0 +1,93 @@
+// pc_internal.h -- context, device tables and launchers shared by the
+// libpc translation units (never exported).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/pc.h"
+
+namespace pc {
+
+typedef uint32_t u32;
+typedef uint64_t u64;
+
+constexpr int MAX_L = 64;       // ciphertext primes
+constexpr int MAX_ALPHA = 8;    // special primes (digit size)
+constexpr int KEYS_PER_LAUNCH = 16;
+
+// Per-prime constants (device).  Shoup companions w' = floor(w 2^32 / q).
+struct PrimeK {
+    u32 q;
+    u32 qn;          // -q^-1 mod 2^32 (REDC)
+    u32 q1s;         // floor(2^32 / q)
+    u32 r32, r32s;   // 2^32 mod q
+    u32 r64, r64s;   // 2^64 mod q
+    u32 ninv, ninvs; // N^-1 mod q
+    u32 pad[7];
+};
+
+// Device tables of one context, passed to kernels by value.
+struct Tables {
+    const PrimeK *pk;        // [NP]
+    const uint2 *colF;       // [NP][R]  psi_rev[k], k < R
+    const uint2 *colI;       // [NP][R]  psi^-1 rev
+    const uint2 *rowF;       // [NP][R][C] per-row re-laid twiddles
+    const uint2 *rowI;       // [NP][R][C]
+    const uint2 *upScale;    // [alpha][L]: N^-1 [Dhat_i^-1]_{q_i}, digit of size d at index d-1
+    const u32 *upConv;       // [dnum][alpha][NP][alpha]: [Dhat_k mod g] 2^32 mod g
+    const uint2 *downScale;  // [alpha]: N^-1 [Phat_k^-1]_{p_k}
+    const u32 *downConv;     // [L][alpha]: [Phat_k mod q_i] 2^32 mod q_i
+    const uint2 *pInv;       // [L]: [P^-1]_{q_i}
+    int *err;                // device error word
+    u32 L, alpha, dnum, NP;
+};
+
+// Up to KEYS_PER_LAUNCH keys, by value in the kernel parameters.
+struct KeyPack {
+    const u32 *b[KEYS_PER_LAUNCH];
+    const u32 *a[KEYS_PER_LAUNCH];
+    u32 seed[KEYS_PER_LAUNCH][8];
+};
+
+}  // namespace pc
+
+struct pc_ctx {
+    int device;
+    int num_sms;
+    uint32_t logN, N, L, alpha, dnum, NP;
+    uint32_t primes[pc::MAX_L + pc::MAX_ALPHA];
+    uint32_t psi[pc::MAX_L + pc::MAX_ALPHA];
+    pc::Tables tab;
+    void *dev_block;  // one allocation holding every table
+    size_t dev_bytes;
+    void *ws;         // caller's workspace
+    size_t ws_bytes;
+    // per-kernel timing (pc_profile_begin / pc_profile_end)
+    cudaEvent_t *prof_ev;   // [prof_max][PC_PROFILE_STAGES + 1]
+    uint32_t prof_max, prof_used;
+};
+
+namespace pc {
+
+// launchers (kernels.cu); each returns a cudaError_t from the launch
+cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
+                       u32 nlimbs, u32 Z, size_t zin, size_t zout, bool canonical, cudaStream_t s);
+// scale_mode: 0 none, 1 N^-1, 2 ModUp digit scale at level l, 3 ModDown P-hat scale
+cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
+                       u32 nlimbs, u32 Z, size_t zin, size_t zout, int scale_mode, u32 l,
+                       cudaStream_t s);
+// mode 0: ModUp (units = digits), 1: ModDown (units = halves)
+cudaError_t launch_bconv_col(const pc_ctx *c, int mode, const u32 *y, size_t yz, u32 *out,
+                             size_t outz, u32 l, u32 Z, cudaStream_t s);
+cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz,
+                         const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l, const KeyPack &kp,
+                         u32 Z, bool regen, bool pintt, cudaStream_t s);
+cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc,
+                               size_t accz, const u32 *c0, size_t c0z, u32 *out0, u32 *out1,
+                               size_t outz, u32 l, u32 Z, cudaStream_t s);
+cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l, cudaStream_t s);
+cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, cudaStream_t s);
+cudaError_t prepare_kernels(const pc_ctx *c);
+
+}  // namespace pc

@@ -1,0 +1,257 @@
+"""Thin ctypes binding of libpc (include/pc.h): argument marshalling only.
+
+Every operation runs in the CUDA library; there is no CPU path.  Device
+buffers are torch CUDA tensors of a 4-byte dtype (int32 or uint32 storage,
+contiguous); they are passed as raw pointers.  If libpc.so is missing the
+import fails with instructions to build it -- it never falls back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpc.so")
+
+PC_OK = 0
+ERRORS = {-1: "PC_E_ARG", -2: "PC_E_ALIGN", -3: "PC_E_CUDA", -4: "PC_E_DEVICE",
+          -5: "PC_E_TIMEOUT", -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE"}
+
+# names of every exported entry point of include/pc.h
+EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_workspace_bytes",
+           "pc_set_workspace", "pc_ntt_fwd", "pc_ntt_inv", "pc_modup", "pc_keyswitch_inner",
+           "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
+           "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end")
+PROFILE_STAGES = ("intt_row_c1", "intt_col_modup_scale", "modup_bconv_col", "inner_chacha",
+                  "moddown_intt_col", "moddown_bconv_col", "moddown_finish")
+
+
+class PCError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {ERRORS.get(code, code)} ({strerror(code)})")
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("logN", ctypes.c_uint32), ("L", ctypes.c_uint32), ("alpha", ctypes.c_uint32),
+                ("dnum", ctypes.c_uint32), ("q", ctypes.POINTER(ctypes.c_uint32)),
+                ("p", ctypes.POINTER(ctypes.c_uint32))]
+
+
+class _Ksk(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint8 * 32), ("b", ctypes.c_void_p), ("a", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libpc.so (built by key_switching_b200.build / __graft_entry__.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m key_switching_b200.build` "
+                              "(the library has no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        u32, i32, vp, sz = ctypes.c_uint32, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+        L.pc_gen_primes.argtypes = [u32, u32, u32, ctypes.POINTER(u32)]
+        L.pc_gen_primes.restype = i32
+        L.pc_ctx_create.argtypes = [ctypes.POINTER(_Params), i32, ctypes.POINTER(vp)]
+        L.pc_ctx_create.restype = i32
+        L.pc_ctx_destroy.argtypes = [vp]
+        L.pc_ctx_destroy.restype = None
+        L.pc_psi.argtypes = [vp, u32]
+        L.pc_psi.restype = u32
+        L.pc_workspace_bytes.argtypes = [vp, u32, u32]
+        L.pc_workspace_bytes.restype = sz
+        L.pc_set_workspace.argtypes = [vp, vp, sz]
+        L.pc_set_workspace.restype = i32
+        for name in ("pc_ntt_fwd", "pc_ntt_inv"):
+            getattr(L, name).argtypes = [vp, vp, u32, u32, u32, vp]
+            getattr(L, name).restype = i32
+        L.pc_modup.argtypes = [vp, vp, u32, vp, vp]
+        L.pc_modup.restype = i32
+        L.pc_keyswitch_inner.argtypes = [vp, vp, u32, ctypes.POINTER(_Ksk), vp, vp]
+        L.pc_keyswitch_inner.restype = i32
+        L.pc_moddown.argtypes = [vp, vp, u32, vp, vp]
+        L.pc_moddown.restype = i32
+        L.pc_keyswitch.argtypes = [vp, vp, vp, u32, ctypes.POINTER(_Ksk), vp, vp, vp]
+        L.pc_keyswitch.restype = i32
+        L.pc_keyswitch_batch.argtypes = [vp, vp, u32, u32, ctypes.POINTER(_Ksk), vp, vp]
+        L.pc_keyswitch_batch.restype = i32
+        L.pc_expand_a.argtypes = [vp, ctypes.c_char_p, u32, vp, vp]
+        L.pc_expand_a.restype = i32
+        L.pc_check.argtypes = [vp]
+        L.pc_check.restype = i32
+        L.pc_strerror.argtypes = [i32]
+        L.pc_strerror.restype = ctypes.c_char_p
+        L.pc_microbench.argtypes = [i32, i32, u32, ctypes.POINTER(ctypes.c_double)]
+        L.pc_microbench.restype = i32
+        L.pc_profile_begin.argtypes = [vp, u32]
+        L.pc_profile_begin.restype = i32
+        L.pc_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(u32)]
+        L.pc_profile_end.restype = i32
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().pc_strerror(code).decode()
+
+
+def _ok(rc: int, what: str):
+    if rc != PC_OK:
+        raise PCError(rc, what)
+
+
+def _ptr(t) -> int:
+    """Raw device pointer of a contiguous 4-byte-element torch tensor (or None)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    assert t.is_cuda and t.is_contiguous() and t.element_size() == 4, "need a contiguous 32-bit CUDA tensor"
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def gen_primes(logN: int, bits: int, count: int):
+    out = (ctypes.c_uint32 * count)()
+    _ok(lib().pc_gen_primes(logN, bits, count, out), "pc_gen_primes")
+    return [int(v) for v in out]
+
+
+def chain(logN: int, bits: int, L: int, alpha: int):
+    """(q, p): the first alpha primes are the special primes, the next L the q's."""
+    pr = gen_primes(logN, bits, L + alpha)
+    return pr[alpha:], pr[:alpha]
+
+
+def microbench(kind: int, iters: int = 4096, device: int = 0) -> float:
+    out = ctypes.c_double()
+    _ok(lib().pc_microbench(device, kind, iters, ctypes.byref(out)), "pc_microbench")
+    return out.value
+
+
+class KSK:
+    """A key-switching key: 32-byte ChaCha12 seed, device 'b' half, optional
+    stored 'a' half (None = regenerate in-kernel)."""
+
+    def __init__(self, seed: bytes, b, a=None):
+        assert len(seed) == 32
+        self.seed, self.b, self.a = bytes(seed), b, a
+
+    def _c(self) -> _Ksk:
+        k = _Ksk()
+        k.seed[:] = list(self.seed)
+        k.b = _ptr(self.b)
+        k.a = _ptr(self.a) if self.a is not None else None
+        return k
+
+
+class Context:
+    """A libpc context on one device: the RNS basis and its device tables."""
+
+    def __init__(self, logN: int, q: Sequence[int], p: Sequence[int], device: int = 0):
+        self.logN, self.N = int(logN), 1 << int(logN)
+        self.q, self.p = [int(v) for v in q], [int(v) for v in p]
+        self.L, self.alpha = len(self.q), len(self.p)
+        self.dnum = -(-self.L // self.alpha)
+        self.device = device
+        qa = (ctypes.c_uint32 * self.L)(*self.q)
+        pa = (ctypes.c_uint32 * self.alpha)(*self.p)
+        prm = _Params(self.logN, self.L, self.alpha, self.dnum, qa, pa)
+        h = ctypes.c_void_p()
+        _ok(lib().pc_ctx_create(ctypes.byref(prm), device, ctypes.byref(h)), "pc_ctx_create")
+        self._h = h
+        self._ws = None
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().pc_ctx_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def prime(self, g: int) -> int:
+        return self.q[g] if g < self.L else self.p[g - self.L]
+
+    def psi(self, g: int) -> int:
+        return int(lib().pc_psi(self._h, g))
+
+    def workspace_bytes(self, l: int, B: int = 1) -> int:
+        return int(lib().pc_workspace_bytes(self._h, l, B))
+
+    def set_workspace(self, buf) -> None:
+        """Hand a device buffer (e.g. a torch uint8/int32 CUDA tensor) to the
+        context; keeps a reference so it outlives the calls that use it."""
+        if buf is None:
+            _ok(lib().pc_set_workspace(self._h, None, 0), "pc_set_workspace")
+        else:
+            _ok(lib().pc_set_workspace(self._h, buf.data_ptr(), buf.numel() * buf.element_size()),
+                "pc_set_workspace")
+        self._ws = buf
+
+    def ensure_workspace(self, l: int, B: int = 1):
+        """Allocate (with torch) and set a workspace big enough for level l, B cts."""
+        import torch
+        need = self.workspace_bytes(l, B)
+        if self._ws is None or self._ws.numel() * self._ws.element_size() < need:
+            self.set_workspace(torch.empty(need, dtype=torch.uint8, device=f"cuda:{self.device}"))
+        return self._ws
+
+    def ntt_fwd(self, x, first_prime: int, nlimbs: int, batch: int = 1, stream=None):
+        _ok(lib().pc_ntt_fwd(self._h, _ptr(x), first_prime, nlimbs, batch, _stream(stream)), "pc_ntt_fwd")
+
+    def ntt_inv(self, x, first_prime: int, nlimbs: int, batch: int = 1, stream=None):
+        _ok(lib().pc_ntt_inv(self._h, _ptr(x), first_prime, nlimbs, batch, _stream(stream)), "pc_ntt_inv")
+
+    def modup(self, c1, l: int, ext, stream=None):
+        _ok(lib().pc_modup(self._h, _ptr(c1), l, _ptr(ext), _stream(stream)), "pc_modup")
+
+    def keyswitch_inner(self, ext, l: int, key: KSK, acc, stream=None):
+        k = key._c()
+        _ok(lib().pc_keyswitch_inner(self._h, _ptr(ext), l, ctypes.byref(k), _ptr(acc), _stream(stream)),
+            "pc_keyswitch_inner")
+
+    def moddown(self, acc, l: int, out, stream=None):
+        _ok(lib().pc_moddown(self._h, _ptr(acc), l, _ptr(out), _stream(stream)), "pc_moddown")
+
+    def keyswitch(self, c0, c1, l: int, key: KSK, c0o, c1o, stream=None):
+        k = key._c()
+        _ok(lib().pc_keyswitch(self._h, _ptr(c0), _ptr(c1), l, ctypes.byref(k), _ptr(c0o), _ptr(c1o),
+                               _stream(stream)), "pc_keyswitch")
+
+    def keyswitch_batch(self, ct, B: int, l: int, keys: Sequence[KSK], out, stream=None):
+        arr = (_Ksk * B)(*[k._c() for k in keys])
+        _ok(lib().pc_keyswitch_batch(self._h, _ptr(ct), B, l, arr, _ptr(out), _stream(stream)),
+            "pc_keyswitch_batch")
+
+    def expand_a(self, seed: bytes, l: int, out, stream=None):
+        _ok(lib().pc_expand_a(self._h, bytes(seed), l, _ptr(out), _stream(stream)), "pc_expand_a")
+
+    def check(self):
+        _ok(lib().pc_check(self._h), "pc_check")
+
+    def profile_begin(self, max_calls: int):
+        _ok(lib().pc_profile_begin(self._h, max_calls), "pc_profile_begin")
+
+    def profile_end(self):
+        """-> (dict stage -> summed ms, number of recorded calls)"""
+        ms = (ctypes.c_float * len(PROFILE_STAGES))()
+        n = ctypes.c_uint32()
+        _ok(lib().pc_profile_end(self._h, ms, ctypes.byref(n)), "pc_profile_end")
+        return dict(zip(PROFILE_STAGES, [float(v) for v in ms])), int(n.value)
