@@ -177,24 +177,29 @@ const char *pc_strerror(int code);
 /* Integer-throughput microbenchmark on `device`: runs `iters` rounds of
  * independent modular-multiply chains (kind 0: Shoup multiply by a constant,
  * the form the NTT and basis conversions use; kind 1: Montgomery multiply of
- * two variables; kind 2: ChaCha12 blocks) over all SMs and writes the
+ * two variables; kind 2: ChaCha12 blocks; kind 3: 32-bit multiply-add; kind
+ * 4: xor + add; kinds 5..8: ChaCha12 blocks with some rotations computed on
+ * the multiply pipe) over all SMs and writes the
  * operations per second to *ops_per_s (modmuls/s, or ChaCha blocks/s).
  * Synchronous.  Returns PC_OK, PC_E_ARG or PC_E_CUDA. */
 int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s);
 
 /* Per-kernel timing of pc_keyswitch / pc_keyswitch_batch, for measurement.
  * pc_profile_begin creates CUDA events (host call, not on the hot path) for up
- * to max_calls key-switch calls; each later call records one event before
- * each of its PC_PROFILE_STAGES kernels and one after the last, on its stream.
- * pc_profile_end synchronises, writes into ms[PC_PROFILE_STAGES] the summed
- * milliseconds of each stage over the recorded calls (stages: 0 inverse row
- * pass of c1, 1 inverse column pass + ModUp scale, 2 ModUp basis conversion +
- * forward column pass, 3 inner product with ChaCha12 + special-limb inverse
- * row pass, 4 special-limb inverse column pass, 5 ModDown basis conversion +
- * forward column pass, 6 ModDown finish), sets *calls, and releases the
- * events.  Returns PC_OK, PC_E_ARG or PC_E_CUDA. */
-#define PC_PROFILE_STAGES 7
-int pc_profile_begin(pc_ctx *ctx, uint32_t max_calls);
+ * to max_calls sampled key-switch calls: of the calls that follow, every
+ * `every`-th one (the 1st, the every+1-th, ...) records one event before each
+ * of its PC_PROFILE_STAGES kernels and one after the last, on its stream;
+ * the others run uninstrumented.  pc_profile_end synchronises, writes into
+ * ms[PC_PROFILE_STAGES] the summed milliseconds of each stage over the
+ * sampled calls (stages: 0 inverse row pass of c1; 1 ModUp column kernel:
+ * inverse column pass + scale, basis conversion, forward column pass;
+ * 2 inner product with ChaCha12 regeneration, forward row pass of the
+ * converted limbs and inverse row pass of the special limbs; 3 ModDown
+ * column kernel; 4 ModDown finish: forward row pass, scale, add), sets *calls
+ * to the number of sampled calls, and releases the events.  Returns PC_OK,
+ * PC_E_ARG or PC_E_CUDA. */
+#define PC_PROFILE_STAGES 5
+int pc_profile_begin(pc_ctx *ctx, uint32_t max_calls, uint32_t every);
 int pc_profile_end(pc_ctx *ctx, float *ms, uint32_t *calls);
 
 #ifdef __cplusplus

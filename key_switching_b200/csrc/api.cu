@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -242,12 +243,22 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
             rowF[base] = make_uint2(0, 0);
             rowI[base] = make_uint2(0, 0);
             for (u32 k = 1; k < C; ++k) {
+                // natural entry k = 2^s + i holds psi_rev[(R + r) 2^s + i]
                 u32 s = 0;
                 while ((2u << s) <= k) ++s;
-                const u32 idx = (R + r) * (1u << s) + (k - (1u << s));
+                const u32 i = k - (1u << s);
+                const u32 idx = (R + r) * (1u << s) + i;
                 const u32 a = rev(pw, idx), b = rev(pwi, idx);
-                rowF[base + k] = make_uint2(a, shoup_of(a, q));
-                rowI[base + k] = make_uint2(b, shoup_of(b, q));
+                // stages s >= 4 (the distance-1 phase): i = (hi << u) + bb is
+                // stored at 2^s + (bb << 4) + hi so a row's threads read
+                // consecutive entries (see TwRow in ntt.cuh)
+                u32 pos = k;
+                if (s >= 4) {
+                    const u32 u = s - 4, hi = i >> u, bb = i & ((1u << u) - 1);
+                    pos = (1u << s) + (bb << 4) + hi;
+                }
+                rowF[base + pos] = make_uint2(a, shoup_of(a, q));
+                rowI[base + pos] = make_uint2(b, shoup_of(b, q));
             }
         }
         pc::PrimeK &K = pk[g];
@@ -356,6 +367,30 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
     T.NP = NP;
     e = pc::prepare_kernels(c);
     if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
+    // Launch attributes.  Programmatic dependent launch lets each kernel stage
+    // its tables while its predecessor drains.  The constant tables are read
+    // by every key switch; an access-policy window marks them persisting in
+    // L2 (within this context's persisting carve-out) so the streamed keys
+    // and ciphertexts do not evict them.
+    c->use_pdl = getenv("PC_NO_PDL") ? 0 : 1;
+    int max_persist = 0, max_window = 0;
+    cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, device);
+    cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, device);
+    if (!getenv("PC_NO_L2_PERSIST") && max_persist > 0 && max_window > 0) {
+        size_t want = total < (size_t)max_persist ? total : (size_t)max_persist;
+        size_t cur = 0;
+        cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize);
+        if (cur < want && cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, want) != cudaSuccess) {
+            cudaGetLastError();
+            want = cur;
+        }
+        if (want > 0) {
+            c->l2_window_base = blk;
+            c->l2_window_bytes = total < (size_t)max_window ? total : (size_t)max_window;
+            const double r = (double)want / (double)c->l2_window_bytes;
+            c->l2_hit_ratio = r >= 1.0 ? 1.0f : (float)r;
+        }
+    }
     *out = c;
     return PC_OK;
 }
@@ -421,8 +456,7 @@ int pc_modup(pc_ctx *c, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream
     const Layout Lw = layout(c, l, 1);
     u32 *w1 = (u32 *)c->ws + Lw.w1;
     cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, s);
-    if (e == cudaSuccess) e = pc::launch_col(c, false, w1, w1, 0, l, 1, 0, 0, 2, l, s);
-    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 0, w1, 0, ext, 0, l, 1, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, s);
     if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
@@ -453,8 +487,7 @@ int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_str
     const size_t N = c->N, ll = l + c->alpha;
     // special-prime limbs of both halves: inverse row pass into the workspace
     cudaError_t e = pc::launch_row(c, false, acc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, false, s);
-    if (e == cudaSuccess) e = pc::launch_col(c, false, wacc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, 3, l, s);
-    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 1, wacc, 2 * ll * N, wu, 2 * l * N, l, 1, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, 2 * ll * N, wu, 2 * l * N, l, 1, s);
     if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, 0, acc, 0, nullptr, 0, out, out + l * N, 0, l, 1, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
@@ -466,21 +499,19 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
     const Layout Lw = layout(c, l, B);
     u32 *ws = (u32 *)c->ws;
     u32 *w1 = ws + Lw.w1, *wt = ws + Lw.t, *wacc = ws + Lw.acc, *wu = ws + Lw.u;
-    const size_t N = c->N, ll = l + c->alpha;
     const bool regen = keys[0].a == nullptr;
     for (u32 b = 1; b < B; ++b)
         if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
     // optional per-stage events (measurement only)
     cudaEvent_t *ev = nullptr;
-    if (c->prof_ev && c->prof_used < c->prof_max) ev = c->prof_ev + (size_t)(c->prof_used++) * (PC_PROFILE_STAGES + 1);
+    if (c->prof_ev && c->prof_used < c->prof_max && (c->prof_seen++ % c->prof_every) == 0)
+        ev = c->prof_ev + (size_t)(c->prof_used++) * (PC_PROFILE_STAGES + 1);
     auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
     mark(0);
     cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, B, cz, Lw.w1z, false, s);
     mark(1);
-    if (e == cudaSuccess) e = pc::launch_col(c, false, w1, w1, 0, l, B, Lw.w1z, Lw.w1z, 2, l, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, Lw.w1z, wt, Lw.tz, l, B, s);
     mark(2);
-    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 0, w1, Lw.w1z, wt, Lw.tz, l, B, s);
-    mark(3);
     for (u32 b0 = 0; e == cudaSuccess && b0 < B; b0 += pc::KEYS_PER_LAUNCH) {
         const u32 nb = (B - b0 < (u32)pc::KEYS_PER_LAUNCH) ? B - b0 : (u32)pc::KEYS_PER_LAUNCH;
         pc::KeyPack kp{};
@@ -492,14 +523,11 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
         e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, c1 + b0 * cz, cz, wacc + b0 * Lw.accz, Lw.accz, l, kp,
                              nb, regen, true, s);
     }
+    mark(3);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, s);
     mark(4);
-    if (e == cudaSuccess)
-        e = pc::launch_col(c, false, wacc + l * N, wacc + l * N, c->L, c->alpha, 2 * B, ll * N, ll * N, 3, l, s);
-    mark(5);
-    if (e == cudaSuccess) e = pc::launch_bconv_col(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, s);
-    mark(6);
     if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, c0, cz, o0, o1, cz, l, B, s);
-    mark(7);
+    mark(5);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
@@ -535,8 +563,8 @@ int pc_expand_a(pc_ctx *c, const uint8_t seed[32], uint32_t l, uint32_t *a_out, 
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
-int pc_profile_begin(pc_ctx *c, uint32_t max_calls) {
-    if (!c || max_calls < 1 || max_calls > 100000) return PC_E_ARG;
+int pc_profile_begin(pc_ctx *c, uint32_t max_calls, uint32_t every) {
+    if (!c || max_calls < 1 || max_calls > 100000 || every < 1) return PC_E_ARG;
     DeviceGuard dg(c->device);
     prof_release(c);
     const size_t n = (size_t)max_calls * (PC_PROFILE_STAGES + 1);
@@ -553,6 +581,8 @@ int pc_profile_begin(pc_ctx *c, uint32_t max_calls) {
     }
     c->prof_max = max_calls;
     c->prof_used = 0;
+    c->prof_every = every;
+    c->prof_seen = 0;
     return PC_OK;
 }
 

@@ -16,15 +16,33 @@ namespace pc {
 
 __device__ __forceinline__ uint32_t rotl32(uint32_t x, int r) { return __funnelshift_l(x, x, r); }
 
-#define PC_QR(a, b, c, d)                  \
-    a += b; d ^= a; d = rotl32(d, 16);     \
-    c += d; b ^= c; b = rotl32(b, 12);     \
-    a += b; d ^= a; d = rotl32(d, 8);      \
-    c += d; b ^= c; b = rotl32(b, 7);
+// Rotation on the integer multiply pipe: for m = 2^r (kept opaque to the
+// compiler), x*m + umulhi(x, m) = (x << r) | (x >> (32 - r)).  Used for some
+// rotations to balance the ALU pipe (xor, funnel shift) against the
+// multiply-add pipe.
+__device__ __forceinline__ uint32_t rotl_mul(uint32_t x, uint32_t m) { return x * m + __umulhi(x, m); }
+
+// Which of the four quarter-round rotations (16, 12, 8, 7) run on the
+// multiply pipe: bit i set -> rotation i uses rotl_mul with mul[i] = 2^r.
+template <int MULMASK>
+struct ChaRot {
+    uint32_t mul[4];
+    __device__ __forceinline__ uint32_t r(int i, uint32_t x) const {
+        const int amt[4] = {16, 12, 8, 7};
+        return ((MULMASK >> i) & 1) ? rotl_mul(x, mul[i]) : rotl32(x, amt[i]);
+    }
+};
+
+#define PC_QR(a, b, c, d)                          \
+    a += b; d ^= a; d = R.r(0, d);                 \
+    c += d; b ^= c; b = R.r(1, b);                 \
+    a += b; d ^= a; d = R.r(2, d);                 \
+    c += d; b ^= c; b = R.r(3, b);
 
 // out[16] = ChaCha12(seed words k[8], counter, g, j)
-__device__ __forceinline__ void chacha12_block(const uint32_t k[8], uint32_t ctr, uint32_t g,
-                                               uint32_t j, uint32_t out[16]) {
+template <int MULMASK = 0>
+__device__ __forceinline__ void chacha12_block(const uint32_t k[8], uint32_t ctr, uint32_t g, uint32_t j,
+                                               uint32_t out[16], const ChaRot<MULMASK> &R = ChaRot<MULMASK>{}) {
     const uint32_t c0 = 0x61707865u, c1 = 0x3320646eu, c2 = 0x79622d32u, c3 = 0x6b206574u;
     uint32_t x0 = c0, x1 = c1, x2 = c2, x3 = c3;
     uint32_t x4 = k[0], x5 = k[1], x6 = k[2], x7 = k[3];

@@ -43,7 +43,8 @@ struct Phase {
         return ((p >> LOGD) << (LOGD + K)) + (m << LOGD) + (p & (D - 1));
     }
 
-    // forward stages; tw(idx) returns {w, w'} for table index idx in [1, M)
+    // forward stages; tw(s, u, hi, b) returns {w, w'} for the table entry
+    // (1 << s) + (hi << u) + b of stage s = S0 + u (see TwNatural / TwRowSm)
     template <class TW>
     __device__ static __forceinline__ void fwd(u32 v[16], int lt, const TW &tw, u32 q) {
 #pragma unroll
@@ -54,7 +55,7 @@ struct Phase {
                 const int hi = pair(lt, g) >> LOGD;
 #pragma unroll
                 for (int b = 0; b < (1 << u); ++b) {
-                    const uint2 w = tw((1 << (S0 + u)) + (hi << u) + b);
+                    const uint2 w = tw(S0 + u, u, hi, b);
 #pragma unroll
                     for (int a = b * (KK >> u); a < b * (KK >> u) + h; ++a)
                         bf_ct(v[g * KK + a], v[g * KK + a + h], w.x, w.y, q);
@@ -73,7 +74,7 @@ struct Phase {
                 const int hi = pair(lt, g) >> LOGD;
 #pragma unroll
                 for (int b = 0; b < (1 << u); ++b) {
-                    const uint2 w = tw((1 << (S0 + u)) + (hi << u) + b);
+                    const uint2 w = tw(S0 + u, u, hi, b);
 #pragma unroll
                     for (int a = b * (KK >> u); a < b * (KK >> u) + h; ++a)
                         bf_gs(v[g * KK + a], v[g * KK + a + h], w.x, w.y, q);
@@ -103,51 +104,102 @@ struct Plan {
     __device__ static __forceinline__ int inv_out(int lt, int r) { return fwd_in(lt, r); }
 };
 
+// Barriers that order a line's shared-memory exchange: a warp barrier when
+// every line's threads sit in one warp (row passes), a CTA barrier, or a
+// named barrier shared by one group of `n` threads (column passes run by
+// independent thread groups).
+struct SyncWarp {
+    __device__ __forceinline__ void operator()() const { __syncwarp(); }
+};
+struct SyncCta {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct SyncGroup {
+    int id, n;  // barrier id (1..15) and thread count (a multiple of 32)
+    __device__ __forceinline__ void operator()() const {
+        asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+    }
+};
+
 // Exchange the registers of phase A's layout into phase B's layout through
 // shared memory.  ADDR(x) gives the word address of element x of the line.
-template <class PA, class PB, class ADDR>
-__device__ __forceinline__ void exchange(u32 v[16], u32 *sm, int lt, const ADDR &addr) {
-    __syncthreads();
+template <class PA, class PB, class SYNC, class ADDR>
+__device__ __forceinline__ void exchange(u32 v[16], u32 *sm, int lt, const ADDR &addr, const SYNC &sync) {
+    sync();
 #pragma unroll
     for (int r = 0; r < 16; ++r) sm[addr(PA::x_of(lt, r))] = v[r];
-    __syncthreads();
+    sync();
 #pragma unroll
     for (int r = 0; r < 16; ++r) v[r] = sm[addr(PB::x_of(lt, r))];
 }
 
 // Full forward line transform: registers enter at Plan::fwd_in positions and
 // leave at Plan::fwd_out positions (lazy values in [0, 2q)).
-template <int LOGM, class ADDR, class TW>
-__device__ __forceinline__ void line_fwd(u32 v[16], u32 *sm, int lt, const ADDR &addr,
-                                         const TW &tw, u32 q) {
+template <int LOGM, class ADDR, class TW, class SYNC>
+__device__ __forceinline__ void line_fwd(u32 v[16], u32 *sm, int lt, const ADDR &addr, const TW &tw, u32 q,
+                                         const SYNC &sync) {
     using PL = Plan<LOGM>;
     PL::P0::fwd(v, lt, tw, q);
     if constexpr (PL::NPH >= 2) {
-        exchange<typename PL::P0, typename PL::P1>(v, sm, lt, addr);
+        exchange<typename PL::P0, typename PL::P1>(v, sm, lt, addr, sync);
         PL::P1::fwd(v, lt, tw, q);
     }
     if constexpr (PL::NPH >= 3) {
-        exchange<typename PL::P1, typename PL::P2>(v, sm, lt, addr);
+        exchange<typename PL::P1, typename PL::P2>(v, sm, lt, addr, sync);
         PL::P2::fwd(v, lt, tw, q);
     }
 }
 
 // Full inverse line transform (no N^-1): registers enter at Plan::inv_in
 // and leave at Plan::inv_out positions.
-template <int LOGM, class ADDR, class TW>
-__device__ __forceinline__ void line_inv(u32 v[16], u32 *sm, int lt, const ADDR &addr,
-                                         const TW &tw, u32 q) {
+template <int LOGM, class ADDR, class TW, class SYNC>
+__device__ __forceinline__ void line_inv(u32 v[16], u32 *sm, int lt, const ADDR &addr, const TW &tw, u32 q,
+                                         const SYNC &sync) {
     using PL = Plan<LOGM>;
     if constexpr (PL::NPH >= 3) {
         PL::P2::inv(v, lt, tw, q);
-        exchange<typename PL::P2, typename PL::P1>(v, sm, lt, addr);
+        exchange<typename PL::P2, typename PL::P1>(v, sm, lt, addr, sync);
     }
     if constexpr (PL::NPH >= 2) {
         PL::P1::inv(v, lt, tw, q);
-        exchange<typename PL::P1, typename PL::P0>(v, sm, lt, addr);
+        exchange<typename PL::P1, typename PL::P0>(v, sm, lt, addr, sync);
     }
     PL::P0::inv(v, lt, tw, q);
 }
+
+// Twiddle tables.  Natural layout: entry (1 << s) + (hi << u) + b.
+struct TwNatural {
+    const uint2 *t;
+    __device__ __forceinline__ uint2 operator()(int s, int u, int hi, int b) const {
+        return t[(1 << s) + (hi << u) + b];
+    }
+};
+// Row tables as stored on the device: stages s >= 4 (the distance-1 phase,
+// where every thread of a row has its own twiddles) are re-laid as
+// (1 << s) + (b << 4) + hi, so that at fixed b the threads of a row read
+// consecutive entries (no shared-memory bank conflicts); stages s < 4 are
+// shared by the whole row (broadcast) and keep the natural layout.
+struct TwRow {
+    const uint2 *t;
+    __device__ __forceinline__ uint2 operator()(int s, int u, int hi, int b) const {
+        return s < 4 ? t[(1 << s) + (hi << u) + b] : t[(1 << s) + (b << 4) + hi];
+    }
+};
+
+// 16-byte asynchronous global -> shared copy (bypasses registers and L1)
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// Programmatic dependent launch: pdl_wait() blocks until the previous grid on
+// the stream has completed and its writes are visible (a no-op when the
+// kernel was launched without the attribute); pdl_trigger() lets the next
+// grid start launching once every CTA of this grid has called it.  Kernels
+// read only constant tables before pdl_wait() and write nothing before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" :::); }
 
 // Geometry of a ring of degree 2^LOGN_: C = 2^LOGC-word rows, R = 2^LOGR rows.
 template <int LOGN_>
@@ -156,18 +208,21 @@ struct Geo {
     static constexpr int LOGC = (LOGN - 4 < 8) ? LOGN - 4 : 8;
     static constexpr int LOGR = LOGN - LOGC;
     static constexpr int N = 1 << LOGN, C = 1 << LOGC, R = 1 << LOGR;
-    // row pass: NL rows per CTA, C/16 threads per row
+    // row pass: NL rows per CTA (64 threads), C/16 threads per row
     static constexpr int TPR = C / 16;
-    static constexpr int NL = (4096 / C < R) ? 4096 / C : R;
+    static constexpr int NL = (64 / TPR < R) ? 64 / TPR : R;
     static constexpr int ROW_THREADS = NL * TPR;
     static constexpr int ROW_BLOCKS = R / NL;
     static constexpr int ROW_LS = C + C / 16;  // padded row stride in shared memory
-    // column pass: W columns per CTA, R/16 threads per column
+    // column pass: W columns per CTA (128..256 threads), R/16 threads per column;
+    // the shared tile is row-major with one W-word pad every 16 rows, which
+    // keeps the phase exchanges free of bank conflicts
     static constexpr int TPCOL = R / 16;
-    static constexpr int W = (4096 / R < C) ? 4096 / R : C;
+    static constexpr int W_ = 2048 / R > 4 ? 2048 / R : 4;
+    static constexpr int W = W_ < C ? W_ : C;
     static constexpr int COL_THREADS = W * TPCOL;
     static constexpr int COL_BLOCKS = C / W;
-    static constexpr int COL_LS = W + 1;  // padded shared-memory row stride of a column tile
+    static constexpr int COL_TILE = (R + R / 16) * W;  // words of the padded tile
     static_assert(LOGC >= 4 && LOGR >= 4 && LOGR <= 9, "supported 2^8..2^17 (R,C >= 16)");
 };
 

@@ -63,9 +63,14 @@ struct pc_ctx {
     size_t dev_bytes;
     void *ws;         // caller's workspace
     size_t ws_bytes;
+    // launch attributes: programmatic dependent launch, L2 persistence of the tables
+    int use_pdl;
+    void *l2_window_base;
+    size_t l2_window_bytes;
+    float l2_hit_ratio;
     // per-kernel timing (pc_profile_begin / pc_profile_end)
     cudaEvent_t *prof_ev;   // [prof_max][PC_PROFILE_STAGES + 1]
-    uint32_t prof_max, prof_used;
+    uint32_t prof_max, prof_used, prof_every, prof_seen;
 };
 
 namespace pc {
@@ -77,9 +82,14 @@ cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 f
 cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
                        u32 nlimbs, u32 Z, size_t zin, size_t zout, int scale_mode, u32 l,
                        cudaStream_t s);
-// mode 0: ModUp (units = digits), 1: ModDown (units = halves)
-cudaError_t launch_bconv_col(const pc_ctx *c, int mode, const u32 *y, size_t yz, u32 *out,
-                             size_t outz, u32 l, u32 Z, cudaStream_t s);
+// fused cluster kernel: inverse column pass + scale of the sources, DSMEM
+// gather, conversion and forward column pass of the targets.  mode 0 (ModUp):
+// src = the inverse-row-pass output of c1 [l][N], out = T [beta][l+alpha][N];
+// mode 1 (ModDown): src = ACC [2][l+alpha][N] (special limbs row-inverted),
+// out = U [2][l][N]
+
+cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz,
+                           u32 l, u32 Z, cudaStream_t s);
 cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz,
                          const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l, const KeyPack &kp,
                          u32 Z, bool regen, bool pintt, cudaStream_t s);

@@ -23,8 +23,7 @@ EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_wor
            "pc_set_workspace", "pc_ntt_fwd", "pc_ntt_inv", "pc_modup", "pc_keyswitch_inner",
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
            "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end")
-PROFILE_STAGES = ("intt_row_c1", "intt_col_modup_scale", "modup_bconv_col", "inner_chacha",
-                  "moddown_intt_col", "moddown_bconv_col", "moddown_finish")
+PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
 class PCError(RuntimeError):
@@ -88,7 +87,7 @@ def lib():
         L.pc_strerror.restype = ctypes.c_char_p
         L.pc_microbench.argtypes = [i32, i32, u32, ctypes.POINTER(ctypes.c_double)]
         L.pc_microbench.restype = i32
-        L.pc_profile_begin.argtypes = [vp, u32]
+        L.pc_profile_begin.argtypes = [vp, u32, u32]
         L.pc_profile_begin.restype = i32
         L.pc_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(u32)]
         L.pc_profile_end.restype = i32
@@ -246,8 +245,8 @@ class Context:
     def check(self):
         _ok(lib().pc_check(self._h), "pc_check")
 
-    def profile_begin(self, max_calls: int):
-        _ok(lib().pc_profile_begin(self._h, max_calls), "pc_profile_begin")
+    def profile_begin(self, max_calls: int, every: int = 1):
+        _ok(lib().pc_profile_begin(self._h, max_calls, every), "pc_profile_begin")
 
     def profile_end(self):
         """-> (dict stage -> summed ms, number of recorded calls)"""

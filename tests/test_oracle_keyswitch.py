@@ -2,11 +2,22 @@
 
 Keygen identity: b_j + a_j*s - [P]_q * g_j * s' recomputed equals e_j exactly
 (coefficient form).  Automorphism: s(X^g) by brute-force substitution.
-Key switch: decryption under the true secret after switching s' -> s matches
-decryption before, within the error bound derived in DESIGN (hybrid key
-switching, Han-Ki 2020):  |err| <= sum_j |D_j| Q_{D_j} ||e_j||_1 / P
-                                   + (1 + alpha)(1 + ||s||_1),
-and a wrong key breaks it (the check has teeth).
+
+Key switch (hybrid key switching, Han-Ki 2020): decryption under the true
+secret after switching s' -> s matches decryption before, within
+
+    B = sum_j |D_j| Q_{D_j} ||e_j||_1 / P + (1 + alpha)(1 + ||s||_1).
+
+Derivation.  Let A_h be the integer lift of acc_h over Q_l P.  With d~_j the
+ModUp value of digit j (0 <= d~_j < |D_j| Q_{D_j}) and b_j + a_j s = e_j +
+P G_j s' (G_j = 1 mod the digit's primes, 0 mod the other q's),
+A_b + A_a s = P c1 s' + E (mod Q_l P), E = sum_j d~_j e_j, because
+sum_j d~_j G_j = c1 (mod Q_l).  ModDown gives out_h = (A_h - r_h)/P - v_h with
+r_h = A_h mod P and 0 <= v_h < alpha.  Hence
+(c0' + c1' s) - (c0 + c1 s') = E/P - (r_b + r_a s)/P - v_b - v_a s (mod Q_l),
+and |E/P| <= sum_j ||d~_j||_inf ||e_j||_1 / P, |r_b/P| < 1, |r_a s/P| < ||s||_1,
+|v_b| < alpha, |v_a s| <= alpha ||s||_1.  A wrong key breaks the bound (teeth),
+and every tested bound is below Q_l/2.
 """
 import numpy as np
 import pytest
