@@ -53,6 +53,7 @@ extern "C" {
 #define PC_E_TIMEOUT (-5)   /* a bounded device wait gave up */
 #define PC_E_PRIME (-6)     /* a modulus is not prime, not = 1 mod 2N, or >= 2^31 */
 #define PC_E_WORKSPACE (-7) /* no workspace set, or smaller than pc_workspace_bytes */
+#define PC_E_TOO_BIG (-8)   /* size beyond the static scratch of pc_modup_noalloc */
 
 typedef struct pc_ctx pc_ctx; /* opaque; owns the device constant tables */
 typedef void *pc_stream;      /* a cudaStream_t */
@@ -126,6 +127,21 @@ int pc_ntt_inv(pc_ctx *ctx, uint32_t *x, uint32_t first_prime, uint32_t nlimbs,
  * digit's other primes; for t not in D_j, ext[j][t] = NTT_t(sum_i y_i [Dhat_i]_t
  * mod t); for t in D_j, ext[j][t] = c1[t].  Needs the workspace. */
 int pc_modup(pc_ctx *ctx, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream stream);
+
+/* pc_modup without a workspace, for callers that cannot allocate device
+ * memory (a plugin inside a host framework that owns every device allocation,
+ * or a latency-critical path that cannot afford cudaMalloc's device-wide
+ * synchronisation).  The pages have no counterpart of this call; it computes
+ * exactly what pc_modup computes, with the same arguments, layouts and status
+ * codes, and needs no pc_set_workspace.  Its l*N words of scratch live in one
+ * statically allocated device array of 2^21 words (8 MiB) that the library
+ * holds on every device it is loaded on until the process exits; l*N above
+ * 2^21 returns PC_E_TOO_BIG.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current) and caches
+ * it, so that first call should be made before any stream capture.  All calls
+ * share the array and it keeps the last call's contents (nothing in it needs
+ * to start at zero); calls whose kernels overlap on the GPU race on it. */
+int pc_modup_noalloc(pc_ctx *ctx, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream stream);
 
 /* Key inner product with in-kernel ChaCha12 regeneration of 'a'.
  * ext: device [beta][l+alpha][N] (pc_modup's output).  acc: device

@@ -158,6 +158,10 @@ void prof_release(pc_ctx *c) {
 
 }  // namespace
 
+namespace pc {
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace pc
+
 extern "C" {
 
 int pc_gen_primes(uint32_t logN, uint32_t bits, uint32_t count, uint32_t *out) {
@@ -631,6 +635,7 @@ const char *pc_strerror(int code) {
         case PC_E_TIMEOUT: return "a bounded device wait gave up";
         case PC_E_PRIME: return "modulus not prime, not 1 mod 2N, repeated, or >= 2^31";
         case PC_E_WORKSPACE: return "workspace missing or smaller than pc_workspace_bytes";
+        case PC_E_TOO_BIG: return "l*N exceeds the static scratch of pc_modup_noalloc (2^21 words)";
         default: return "unknown status code";
     }
 }

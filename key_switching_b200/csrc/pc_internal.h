@@ -100,4 +100,7 @@ cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l,
 cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, cudaStream_t s);
 cudaError_t prepare_kernels(const pc_ctx *c);
 
+// Remember a CUDA error for pc_strerror(PC_E_CUDA); returns PC_E_CUDA.
+int record_cuda_error(cudaError_t e);
+
 }  // namespace pc

@@ -16,13 +16,13 @@ LIB_PATH = os.path.join(_HERE, "libpc.so")
 
 PC_OK = 0
 ERRORS = {-1: "PC_E_ARG", -2: "PC_E_ALIGN", -3: "PC_E_CUDA", -4: "PC_E_DEVICE",
-          -5: "PC_E_TIMEOUT", -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE"}
+          -5: "PC_E_TIMEOUT", -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE", -8: "PC_E_TOO_BIG"}
 
 # names of every exported entry point of include/pc.h
 EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_workspace_bytes",
            "pc_set_workspace", "pc_ntt_fwd", "pc_ntt_inv", "pc_modup", "pc_keyswitch_inner",
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
-           "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end")
+           "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
@@ -91,6 +91,8 @@ def lib():
         L.pc_profile_begin.restype = i32
         L.pc_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(u32)]
         L.pc_profile_end.restype = i32
+        L.pc_modup_noalloc.argtypes = [vp, vp, u32, vp, vp]
+        L.pc_modup_noalloc.restype = i32
         _lib = L
     return _lib
 
@@ -220,6 +222,11 @@ class Context:
 
     def modup(self, c1, l: int, ext, stream=None):
         _ok(lib().pc_modup(self._h, _ptr(c1), l, _ptr(ext), _stream(stream)), "pc_modup")
+
+    def modup_noalloc(self, c1, l: int, ext, stream=None):
+        """pc_modup with its scratch in the library's static device array
+        (no workspace; for callers that cannot allocate device memory)."""
+        _ok(lib().pc_modup_noalloc(self._h, _ptr(c1), l, _ptr(ext), _stream(stream)), "pc_modup_noalloc")
 
     def keyswitch_inner(self, ext, l: int, key: KSK, acc, stream=None):
         k = key._c()
