@@ -237,10 +237,18 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
             pwi[k] = mulm(pwi[k - 1], psii, q);
         }
         auto rev = [&](const std::vector<u32> &t, u32 k) { return t[brv(k, P->logN)]; };
+        // re-laid position of natural table entry k (see TwRow in ntt.cuh)
+        auto relay = [](u32 k) -> u32 {
+            if (k == 0) return 0;
+            u32 s = 0;
+            while ((2u << s) <= k) ++s;
+            const u32 i = k - (1u << s), u = s & 3u, s0 = s - u;
+            return (1u << s) + ((i & ((1u << u) - 1)) << s0) + (i >> u);
+        };
         for (u32 k = 0; k < R; ++k) {
             const u32 a = rev(pw, k), b = rev(pwi, k);
-            colF[(size_t)g * R + k] = make_uint2(a, shoup_of(a, q));
-            colI[(size_t)g * R + k] = make_uint2(b, shoup_of(b, q));
+            colF[(size_t)g * R + relay(k)] = make_uint2(a, shoup_of(a, q));
+            colI[(size_t)g * R + relay(k)] = make_uint2(b, shoup_of(b, q));
         }
         for (u32 r = 0; r < R; ++r) {
             const size_t base = (size_t)g * N + (size_t)r * C;
@@ -253,16 +261,8 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
                 const u32 i = k - (1u << s);
                 const u32 idx = (R + r) * (1u << s) + i;
                 const u32 a = rev(pw, idx), b = rev(pwi, idx);
-                // stages s >= 4 (the distance-1 phase): i = (hi << u) + bb is
-                // stored at 2^s + (bb << 4) + hi so a row's threads read
-                // consecutive entries (see TwRow in ntt.cuh)
-                u32 pos = k;
-                if (s >= 4) {
-                    const u32 u = s - 4, hi = i >> u, bb = i & ((1u << u) - 1);
-                    pos = (1u << s) + (bb << 4) + hi;
-                }
-                rowF[base + pos] = make_uint2(a, shoup_of(a, q));
-                rowI[base + pos] = make_uint2(b, shoup_of(b, q));
+                rowF[base + relay(k)] = make_uint2(a, shoup_of(a, q));
+                rowI[base + relay(k)] = make_uint2(b, shoup_of(b, q));
             }
         }
         pc::PrimeK &K = pk[g];
@@ -377,6 +377,15 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
     // L2 (within this context's persisting carve-out) so the streamed keys
     // and ciphertexts do not evict them.
     c->use_pdl = getenv("PC_NO_PDL") ? 0 : 1;
+    {
+        int lo_pri = 0, hi_pri = 0;
+        cudaDeviceGetStreamPriorityRange(&lo_pri, &hi_pri);
+        e = cudaStreamCreateWithPriority(&c->aux, cudaStreamNonBlocking, hi_pri);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming);
+        if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
+        c->overlap = getenv("PC_NO_OVERLAP") ? 0 : 1;
+    }
     int max_persist = 0, max_window = 0;
     cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, device);
     cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, device);
@@ -403,6 +412,9 @@ void pc_ctx_destroy(pc_ctx *c) {
     if (!c) return;
     DeviceGuard dg(c->device);
     prof_release(c);
+    if (c->aux) cudaStreamDestroy(c->aux);
+    if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+    if (c->ev_join) cudaEventDestroy(c->ev_join);
     if (c->dev_block) cudaFree(c->dev_block);
     delete c;
 }
@@ -429,8 +441,8 @@ int pc_ntt_fwd(pc_ctx *c, uint32_t *x, uint32_t first_prime, uint32_t nlimbs, ui
     DeviceGuard dg(c->device);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t z = (size_t)nlimbs * c->N;
-    cudaError_t e = pc::launch_col(c, true, x, x, first_prime, nlimbs, batch, z, z, 0, 0, s);
-    if (e == cudaSuccess) e = pc::launch_row(c, true, x, x, first_prime, nlimbs, batch, z, z, true, s);
+    cudaError_t e = pc::launch_col(c, true, x, x, first_prime, nlimbs, batch, z, z, 0, s);
+    if (e == cudaSuccess) e = pc::launch_row(c, true, x, x, first_prime, nlimbs, batch, z, z, true, false, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
@@ -441,8 +453,8 @@ int pc_ntt_inv(pc_ctx *c, uint32_t *x, uint32_t first_prime, uint32_t nlimbs, ui
     DeviceGuard dg(c->device);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t z = (size_t)nlimbs * c->N;
-    cudaError_t e = pc::launch_row(c, false, x, x, first_prime, nlimbs, batch, z, z, false, s);
-    if (e == cudaSuccess) e = pc::launch_col(c, false, x, x, first_prime, nlimbs, batch, z, z, 1, 0, s);
+    cudaError_t e = pc::launch_row(c, false, x, x, first_prime, nlimbs, batch, z, z, false, false, s);
+    if (e == cudaSuccess) e = pc::launch_col(c, false, x, x, first_prime, nlimbs, batch, z, z, 1, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
@@ -459,8 +471,8 @@ int pc_modup(pc_ctx *c, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream
     cudaStream_t s = (cudaStream_t)stream;
     const Layout Lw = layout(c, l, 1);
     u32 *w1 = (u32 *)c->ws + Lw.w1;
-    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, s);
-    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, s);
+    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, true, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, false, s);
     if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
@@ -490,8 +502,9 @@ int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_str
     u32 *wacc = (u32 *)c->ws + Lw.acc, *wu = (u32 *)c->ws + Lw.u;
     const size_t N = c->N, ll = l + c->alpha;
     // special-prime limbs of both halves: inverse row pass into the workspace
-    cudaError_t e = pc::launch_row(c, false, acc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, false, s);
-    if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, 2 * ll * N, wu, 2 * l * N, l, 1, s);
+    cudaError_t e =
+        pc::launch_row(c, false, acc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, false, true, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, 2 * ll * N, wu, 2 * l * N, l, 1, true, s);
     if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, 0, acc, 0, nullptr, 0, out, out + l * N, 0, l, 1, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
@@ -512,23 +525,42 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
         ev = c->prof_ev + (size_t)(c->prof_used++) * (PC_PROFILE_STAGES + 1);
     auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
     mark(0);
-    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, B, cz, Lw.w1z, false, s);
+    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, B, cz, Lw.w1z, false, true, s);
     mark(1);
-    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, Lw.w1z, wt, Lw.tz, l, B, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, Lw.w1z, wt, Lw.tz, l, B, true, s);
     mark(2);
-    for (u32 b0 = 0; e == cudaSuccess && b0 < B; b0 += pc::KEYS_PER_LAUNCH) {
-        const u32 nb = (B - b0 < (u32)pc::KEYS_PER_LAUNCH) ? B - b0 : (u32)pc::KEYS_PER_LAUNCH;
-        pc::KeyPack kp{};
-        for (u32 i = 0; i < nb; ++i) {
-            kp.b[i] = keys[b0 + i].b;
-            kp.a[i] = keys[b0 + i].a;
-            seed_words(keys[b0 + i].seed, kp.seed[i]);
+    // The ModDown branch needs only the special-prime accumulators: when not
+    // instrumented, those inner products run first on the high-priority
+    // internal stream, followed there by the ModDown conversion kernel, while
+    // the ciphertext-prime inner products run on the caller's stream; the
+    // final kernel joins both.
+    const bool fork = c->overlap && !ev;
+    auto inner = [&](cudaStream_t st, u32 t0, u32 nt) {
+        for (u32 b0 = 0; e == cudaSuccess && b0 < B; b0 += pc::KEYS_PER_LAUNCH) {
+            const u32 nb = (B - b0 < (u32)pc::KEYS_PER_LAUNCH) ? B - b0 : (u32)pc::KEYS_PER_LAUNCH;
+            pc::KeyPack kp{};
+            for (u32 i = 0; i < nb; ++i) {
+                kp.b[i] = keys[b0 + i].b;
+                kp.a[i] = keys[b0 + i].a;
+                seed_words(keys[b0 + i].seed, kp.seed[i]);
+            }
+            e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, c1 + b0 * cz, cz, wacc + b0 * Lw.accz, Lw.accz, l,
+                                 kp, nb, regen, true, st, t0, nt);
         }
-        e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, c1 + b0 * cz, cz, wacc + b0 * Lw.accz, Lw.accz, l, kp,
-                             nb, regen, true, s);
+    };
+    if (fork) {
+        if (e == cudaSuccess) e = cudaEventRecord(c->ev_fork, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(c->aux, c->ev_fork, 0);
+        inner(c->aux, l, c->alpha);
+        if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, true, c->aux);
+        if (e == cudaSuccess) e = cudaEventRecord(c->ev_join, c->aux);
+        inner(s, 0, l);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, c->ev_join, 0);
+    } else {
+        inner(s, 0, 0);
+        mark(3);
+        if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, true, s);
     }
-    mark(3);
-    if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, s);
     mark(4);
     if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, c0, cz, o0, o1, cz, l, B, s);
     mark(5);

@@ -1,23 +1,27 @@
 // kernels.cu -- the key-switching kernels for sm_100a and their launchers.
 //
 // Dataflow of one key switch at level l (hybrid key switching, Han-Ki 2020;
-// full-RNS CKKS, Cheon et al. 2018), with N = R x C (rows of C words):
-//   k_row(inv)         c1 rows: inverse row pass                 -> W1
-//   k_colconv(ModUp)   per digit j and column block, one CTA cluster:
-//                      inverse column pass of the digit's limbs, times
-//                      N^-1 [Dhat_i^-1]_{q_i} (y), shared over DSMEM;
-//                      z_t = sum_i y_i [Dhat_i]_t for t outside D_j,
-//                      forward column pass                        -> T[j][t]
-//   k_inner            per target limb t: forward row pass of T[j][t] (or the
-//                      input limb when t is in D_j), times b_{j,t} and the
-//                      ChaCha12-regenerated a_{j,t}, summed over j; the
-//                      special-prime limbs then get the inverse row pass -> ACC
-//   k_colconv(ModDown) per half and column block: inverse column pass of the
-//                      special limbs times N^-1 [Phat_p^-1]_p, DSMEM share,
-//                      z_i = sum_p y_p [Phat_p]_{q_i}, forward column pass -> U
-//   k_moddown_row      forward row pass of U, (acc - z) [P^-1]_{q_i} (+ c0) -> out
-// Values between passes are lazy ([0, 2q)); every stored result of an ABI call
-// is canonical.
+// full-RNS CKKS, Cheon et al. 2018), with N = R x C viewed as R rows of C
+// words.  The intermediates between a row pass and a column pass are stored
+// column-major ("CM": element (r, c) at c*R + r) so that every column is
+// contiguous; row kernels transpose through a shared-memory tile.
+//   k_row(inv, CM out)  inverse row pass of c1                         -> W1 (CM)
+//   k_colconv(ModUp)    per digit j and 2-column strip: warp k runs the
+//                       inverse column pass of limb k of D_j times
+//                       N^-1 [Dhat_k^-1]; the warps then convert to every
+//                       target t outside D_j (z_t = sum_k y_k [Dhat_k]_t) and
+//                       run its forward column pass                    -> T (CM)
+//   k_inner             per target limb t and 8-row block: forward row pass
+//                       of T[j][t] (or the input limb when t is in D_j), times
+//                       b_{j,t} and the ChaCha12-regenerated a_{j,t}, summed
+//                       over j; special-prime limbs then get the inverse row
+//                       pass                                             -> ACC
+//   k_colconv(ModDown)  per half and strip: inverse column pass of the
+//                       special limbs times N^-1 [Phat_p^-1], conversion to
+//                       every q_i, forward column pass                   -> U (CM)
+//   k_moddown_row       forward row pass of U, (acc - z) [P^-1] (+ c0)   -> out
+// Values between passes are lazy ([0, 2q)); every stored result of an ABI
+// call is canonical.
 #include <cuda_runtime.h>
 
 #include <cooperative_groups.h>
@@ -92,23 +96,65 @@ __device__ __forceinline__ void stage_row_tw(uint2 *stw, const uint2 *tab_rows) 
         cp_async16(stw + 2 * i, tab_rows + 2 * i);
 }
 
+// Column-major staging tile of a row block (NL = 8 rows): for each of the C
+// columns, the block's 8 words as two 16-byte chunks, the chunk order
+// flipped on every other group of 4 columns so that a row's threads writing
+// consecutive columns spread over the banks.
+__device__ __forceinline__ int cm_addr(int x, int rho) {
+    return x * 8 + (((rho >> 2) ^ ((x >> 2) & 1)) << 2) + (rho & 3);
+}
+__device__ __forceinline__ int cm_chunk(int x, int h) { return x * 8 + ((h ^ ((x >> 2) & 1)) << 2); }
+
+// Asynchronously copy the 8 rows [row0, row0+8) of a column-major limb
+// (column x at x*R) into a staging tile.  Caller commits / waits.
 template <class GE>
-constexpr size_t row_smem_bytes() {
-    return sizeof(u32) * GE::NL * GE::ROW_LS + sizeof(uint2) * GE::NL * GE::C;
+__device__ __forceinline__ void stage_cm_rows(u32 *tile, const u32 *limb_cm, int row0) {
+    static_assert(GE::NL == 8, "column-major row blocks are 8 rows (32-byte column segments)");
+    constexpr int CHUNKS = 2 * GE::C;
+#pragma unroll
+    for (int i = 0; i < CHUNKS / GE::ROW_THREADS; ++i) {
+        const int e = threadIdx.x + i * GE::ROW_THREADS;
+        const int x = e >> 1, h = e & 1;
+        cp_async16(tile + cm_chunk(x, h), limb_cm + (size_t)x * GE::R + row0 + 4 * h);
+    }
+}
+
+// Write a staging tile (filled through cm_addr) to the 8 rows [row0, row0+8)
+// of a column-major limb, 16 bytes per access.  Caller synchronises first.
+template <class GE>
+__device__ __forceinline__ void store_cm_rows(const u32 *tile, u32 *limb_cm, int row0) {
+    constexpr int CHUNKS = 2 * GE::C;
+#pragma unroll
+    for (int i = 0; i < CHUNKS / GE::ROW_THREADS; ++i) {
+        const int e = threadIdx.x + i * GE::ROW_THREADS;
+        const int x = e >> 1, h = e & 1;
+        *reinterpret_cast<uint4 *>(limb_cm + (size_t)x * GE::R + row0 + 4 * h) =
+            *reinterpret_cast<const uint4 *>(tile + cm_chunk(x, h));
+    }
+}
+
+// Shared memory of the row kernels: twiddles [NL][C] uint2, exchange lines
+// [NL][ROW_LS], `tiles` column-major staging tiles of C*8 words.
+template <class GE>
+constexpr size_t row_smem_bytes(int tiles) {
+    return sizeof(uint2) * GE::NL * GE::C + sizeof(u32) * (GE::NL * GE::ROW_LS + (size_t)tiles * GE::C * 8);
 }
 
 // ------------------------------------------------------------------ row pass
-// grid (ROW_BLOCKS, nlimbs, Z).  In place allowed (in == out).
-template <int LOGN, bool FWD>
+// grid (ROW_BLOCKS, nlimbs, Z).  Row-major limbs in.  Out: row-major (in
+// place allowed), or for CMOUT (inverse only) column-major limbs.
+template <int LOGN, bool FWD, bool CMOUT>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS)
 k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int canonical) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
     using PLAST = typename LastPhase<GE::LOGC>::type;
+    static_assert(!(CMOUT && FWD), "column-major output is for the inverse pass");
     extern __shared__ __align__(16) u32 dyn[];
-    uint2 *stw = reinterpret_cast<uint2 *>(dyn);          // [NL][C]
-    u32 *sm = dyn + 2 * GE::NL * GE::C;                      // [NL][ROW_LS]
+    uint2 *stw = reinterpret_cast<uint2 *>(dyn);  // [NL][C]
+    u32 *sm = dyn + 2 * GE::NL * GE::C;             // [NL][ROW_LS]
+    u32 *tile = sm + GE::NL * GE::ROW_LS;           // [C][8]
     const int rho = threadIdx.x / GE::TPR, lt = threadIdx.x % GE::TPR;
     const int row0 = blockIdx.x * GE::NL, row = row0 + rho;
     const u32 g = first_prime + blockIdx.y;
@@ -116,9 +162,9 @@ k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
     stage_row_tw<GE>(stw, (FWD ? T.rowF : T.rowI) + (size_t)g * GE::N + (size_t)row0 * GE::C);
     pdl_wait();
     pdl_trigger();
-    const size_t off = (size_t)blockIdx.y * GE::N + (size_t)row * GE::C;
-    const u32 *src = in + blockIdx.z * zin + off;
-    u32 *dst = out + blockIdx.z * zout + off;
+    const size_t limb = (size_t)blockIdx.y * GE::N;
+    const u32 *src = in + blockIdx.z * zin + limb + (size_t)row * GE::C;
+    u32 *dst = out + blockIdx.z * zout + limb;
     u32 v[16];
     u32 *line = sm + rho * GE::ROW_LS;
     const TwRow tw{stw + rho * GE::C};
@@ -126,30 +172,30 @@ k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
     else gload<PLAST>(v, src, lt);
     cp_async_wait_all();
     __syncthreads();
-    if constexpr (FWD) {
-        line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
-        if (canonical) {
+    if constexpr (FWD) line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
+    else line_inv<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
+    if (canonical) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) v[r] = red1(v[r], q);
-        }
-        gstore<PLAST>(v, dst, lt);
+        for (int r = 0; r < 16; ++r) v[r] = red1(v[r], q);
+    }
+    if constexpr (CMOUT) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) tile[cm_addr(PF::x_of(lt, r), rho)] = v[r];
+        __syncthreads();
+        store_cm_rows<GE>(tile, dst, row0);
+    } else if constexpr (FWD) {
+        gstore<PLAST>(v, dst + (size_t)row * GE::C, lt);
     } else {
-        line_inv<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
-        if (canonical) {
-#pragma unroll
-            for (int r = 0; r < 16; ++r) v[r] = red1(v[r], q);
-        }
-        gstore<PF>(v, dst, lt);
+        gstore<PF>(v, dst + (size_t)row * GE::C, lt);
     }
 }
 
-// --------------------------------------------------------------- column pass
-// grid (COL_BLOCKS, nlimbs, Z).  In place allowed.  scale_mode: 0 none (lazy
-// out), 1 N^-1, 2 ModUp digit scale at level l, 3 ModDown P-hat scale.
+// -------------------------------------------- column pass, row-major limbs
+// (the NTT calls).  grid (COL_BLOCKS, nlimbs, Z).  In place allowed.
+// scale_mode 0: lazy output; 1: times N^-1, canonical.
 template <int LOGN, bool FWD>
 __global__ void __launch_bounds__(Geo<LOGN>::COL_THREADS)
-k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int scale_mode,
-      u32 l) {
+k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int scale_mode) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
     using PF = typename PL::P0;
@@ -172,61 +218,48 @@ k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
     if constexpr (FWD) {
 #pragma unroll
         for (int r = 0; r < 16; ++r) v[r] = src[(size_t)PF::x_of(lt, r) * GE::C];
-        line_fwd<GE::LOGR>(v, sm, lt, ColAddr<GE::W>{c}, TwNatural{tw}, q, SyncCta{});
+        line_fwd<GE::LOGR>(v, sm, lt, ColAddr<GE::W>{c}, TwRow{tw}, q, SyncCta{});
 #pragma unroll
         for (int r = 0; r < 16; ++r) dst[(size_t)PLAST::x_of(lt, r) * GE::C] = v[r];
     } else {
 #pragma unroll
         for (int r = 0; r < 16; ++r) v[r] = src[(size_t)PLAST::x_of(lt, r) * GE::C];
-        line_inv<GE::LOGR>(v, sm, lt, ColAddr<GE::W>{c}, TwNatural{tw}, q, SyncCta{});
-        uint2 s = make_uint2(0, 0);
-        if (scale_mode == 1) s = make_uint2(T.pk[g].ninv, T.pk[g].ninvs);
-        else if (scale_mode == 2) {
-            const u32 j = k / T.alpha, d = min(T.alpha, l - j * T.alpha);
-            s = T.upScale[(size_t)(d - 1) * T.L + k];
-        } else if (scale_mode == 3) s = T.downScale[g - T.L];
-        if (scale_mode) {
+        line_inv<GE::LOGR>(v, sm, lt, ColAddr<GE::W>{c}, TwRow{tw}, q, SyncCta{});
+        if (scale_mode == 1) {
+            const u32 s = T.pk[g].ninv, ss = T.pk[g].ninvs;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) v[r] = shoup(v[r], s.x, s.y, q);
+            for (int r = 0; r < 16; ++r) v[r] = shoup(v[r], s, ss, q);
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) dst[(size_t)PF::x_of(lt, r) * GE::C] = v[r];
     }
 }
 
-// ---------------------------------------- fused column kernel (cluster)
-// One cluster of alpha CTAs owns one (unit, column block): CTA k runs the
-// inverse column pass of source limb k (input: the inverse row pass output),
-// multiplies by its conversion scale and leaves the tile y_k in its shared
-// memory; after a cluster barrier every CTA gathers all y tiles over
-// distributed shared memory, then converts them to its share of the target
-// primes (z_t = sum_k y_k c_{k,t}) and runs the forward column pass of each.
-//   mode 0 (ModUp):   unit = digit j, sources q_{j alpha + k} (k < d),
-//                     scale N^-1 [Dhat^-1], targets t not in D_j -> out[j][t]
-//   mode 1 (ModDown): unit = half h, sources p_k (k < alpha),
-//                     scale N^-1 [Phat_k^-1], targets q_i (i < l) -> out[h][i]
-// grid (alpha * COL_BLOCKS, 1, units * Z), cluster (alpha, 1, 1).
-namespace cgx = cooperative_groups;
-
-// Conversion + forward column pass for targets t0 + grp, t0 + grp + NG, ...
-// (NG groups of COL_THREADS threads run their targets concurrently).
-template <int LOGN, int D>
-__device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *out, size_t outz, u32 l,
-                                                u32 unit, u32 z, u32 t0, u32 t1, const u32 *sy, u32 *sx,
-                                                const uint2 *twt, int grp, int NG) {
+// ------------------------------------------------- column conversion kernel
+// One CTA of alpha warps per (unit, strip of CPW columns); a column is held
+// by TPCOL consecutive lanes, so every exchange is warp-synchronous.
+//   mode 0 (ModUp):   unit = digit j; warp k < d runs the inverse column pass
+//                     of limb q_{j alpha + k} (column-major input) times
+//                     N^-1 [Dhat_k^-1]; targets t not in D_j -> out[j][t]
+//   mode 1 (ModDown): unit = half h; warp k runs the inverse column pass of
+//                     special limb k of ACC half h times N^-1 [Phat_k^-1];
+//                     targets q_i, i < l -> out[h][i]
+// The warps then share the y tiles through shared memory and take the
+// targets round-robin: z_t = sum_k y_k [hat_k]_t (Montgomery constants, one
+// REDC), forward column pass, store (column-major, or row-major for OUT_CM
+// false).  grid (C / CPW, 1, units * Z), block 32 * alpha.
+template <int LOGN, int D, bool OUT_CM>
+__device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *out, size_t outz, u32 l, u32 unit,
+                                                u32 z, u32 ntarg, const u32 *sy, u32 *xl0, u32 *xl1, int c, int lt,
+                                                int col) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
     using PF = typename PL::P0;
     using PLAST = typename LastPhase<GE::LOGR>::type;
-    const int tid = threadIdx.x % GE::COL_THREADS;
-    const int c = tid % GE::W, lt = tid / GE::W;
-    const int col0 = (blockIdx.x / T.alpha) * GE::W;
     const u32 ll = l + T.alpha;
-    const SyncGroup gsync{1 + grp, GE::COL_THREADS};
-    for (u32 ti = t0 + grp; ti < t1; ti += NG) {
-        u32 g;
-        const u32 *conv;
-        u32 *dst;
+    const u32 warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
+    // target ti -> (prime, conversion constants, output limb)
+    auto target = [&](u32 ti, u32 &g, const u32 *&conv, u32 *&dst) {
         if (mode == 0) {
             const u32 lo = unit * T.alpha;
             const u32 t = ti < lo ? ti : ti + D;
@@ -238,50 +271,79 @@ __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *
             conv = T.downConv + (size_t)ti * T.alpha;
             dst = out + z * outz + ((size_t)unit * l + ti) * GE::N;
         }
-        const u32 q = T.pk[g].q, qn = T.pk[g].qn, q1s = T.pk[g].q1s;
-        u32 cv[D];
+    };
+    // two targets per warp at a time: ti and ti + nwarps
+    for (u32 ti = warp; ti < ntarg; ti += 2 * nwarps) {
+        const u32 tj = ti + nwarps;
+        const bool two = tj < ntarg;
+        u32 g0, g1;
+        const u32 *conv0, *conv1;
+        u32 *dst0, *dst1;
+        target(ti, g0, conv0, dst0);
+        target(two ? tj : ti, g1, conv1, dst1);
+        const u32 q0 = T.pk[g0].q, qn0 = T.pk[g0].qn, q1s0 = T.pk[g0].q1s;
+        const u32 q1 = T.pk[g1].q, qn1 = T.pk[g1].qn, q1s1 = T.pk[g1].q1s;
+        u32 cv0[D], cv1[D];
 #pragma unroll
-        for (int k = 0; k < D; ++k) cv[k] = __ldg(conv + k);
-        u32 v[16];
+        for (int k = 0; k < D; ++k) {
+            cv0[k] = __ldg(conv0 + k);
+            cv1[k] = __ldg(conv1 + k);
+        }
+        u32 v0[16], v1[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int x = PF::x_of(lt, r);
-            u64 acc = 0;
+            const int xa = c * GE::COL_LS + x + (x >> 4);
+            u64 a0 = 0, a1 = 0;
 #pragma unroll
             for (int k = 0; k < D; ++k) {
-                if (k == 4 || k == 6) acc = fold64(acc, q, q1s);
-                acc += (u64)sy[(k * GE::R + x) * GE::W + c] * cv[k];
+                if (k == 4 || k == 6) {
+                    a0 = fold64(a0, q0, q1s0);
+                    a1 = fold64(a1, q1, q1s1);
+                }
+                const u32 y = sy[k * GE::CPW * GE::COL_LS + xa];
+                a0 += (u64)y * cv0[k];
+                a1 += (u64)y * cv1[k];
             }
-            if constexpr (D <= 4) v[r] = redc((u32)acc, red1((u32)(acc >> 32), q), q, qn);
-            else v[r] = redc64(acc, q, qn, q1s);
+            if constexpr (D <= 4) {
+                v0[r] = redc((u32)a0, red1((u32)(a0 >> 32), q0), q0, qn0);
+                v1[r] = redc((u32)a1, red1((u32)(a1 >> 32), q1), q1, qn1);
+            } else {
+                v0[r] = redc64(a0, q0, qn0, q1s0);
+                v1[r] = redc64(a1, q1, qn1, q1s1);
+            }
         }
-        line_fwd<GE::LOGR>(v, sx + (size_t)grp * GE::COL_TILE, lt, ColAddr<GE::W>{c},
-                           TwNatural{twt + (size_t)(ti - t0) * GE::R}, q, gsync);
+        line_fwd2<GE::LOGR>(v0, v1, xl0, xl1, lt, RowAddr{}, TwRowG{T.colF + (size_t)g0 * GE::R},
+                            TwRowG{T.colF + (size_t)g1 * GE::R}, q0, q1, SyncWarp{});
+        if constexpr (OUT_CM) {
+            gstore<PLAST>(v0, dst0 + (size_t)col * GE::R, lt);
+            if (two) gstore<PLAST>(v1, dst1 + (size_t)col * GE::R, lt);
+        } else {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) dst[(size_t)PLAST::x_of(lt, r) * GE::C + col0 + c] = v[r];
+            for (int r = 0; r < 16; ++r) dst0[(size_t)PLAST::x_of(lt, r) * GE::C + col] = v0[r];
+            if (two) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) dst1[(size_t)PLAST::x_of(lt, r) * GE::C + col] = v1[r];
+            }
+        }
     }
 }
 
-template <int LOGN>
-__global__ void __launch_bounds__(1024)
-k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l, u32 tpc) {
+template <int LOGN, bool OUT_CM>
+__global__ void __launch_bounds__(32 * MAX_ALPHA)
+k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
     using PF = typename PL::P0;
     using PLAST = typename LastPhase<GE::LOGR>::type;
-    cgx::cluster_group cluster = cgx::this_cluster();
     extern __shared__ __align__(16) u32 dyn[];
-    constexpr int TILE = GE::R * GE::W;
-    const int NG = blockDim.x / GE::COL_THREADS;     // concurrent target groups
-    const int grp = threadIdx.x / GE::COL_THREADS, tid = threadIdx.x % GE::COL_THREADS;
-    u32 *own = dyn;                                  // [R][W] this CTA's y tile
-    u32 *sy = own + TILE;                            // [alpha][R][W] gathered tiles
-    u32 *sx = sy + T.alpha * TILE;                   // [NG] padded exchange tiles
-    uint2 *twi = reinterpret_cast<uint2 *>(sx + (size_t)NG * GE::COL_TILE);  // [R] inverse twiddles
-    uint2 *twt = twi + GE::R;                                               // [tpc][R] forward twiddles
-    const u32 rank = cluster.block_rank();
-    const int c = tid % GE::W, lt = tid / GE::W;
-    const int col0 = (blockIdx.x / T.alpha) * GE::W;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int c = lane / GE::TPCOL, lt = lane % GE::TPCOL;
+    const int col = blockIdx.x * GE::CPW + c;
+    u32 *sy = dyn;                                          // [alpha][CPW][COL_LS] y tiles
+    // two exchange lines per warp and column
+    u32 *xl = dyn + (T.alpha + 2 * warp) * GE::CPW * GE::COL_LS + c * GE::COL_LS;
+    u32 *xl1 = xl + GE::CPW * GE::COL_LS;
     const u32 units = mode == 0 ? (l + T.alpha - 1) / T.alpha : 2;
     const u32 z = blockIdx.z / units, unit = blockIdx.z % units;
     const u32 ll = l + T.alpha;
@@ -291,86 +353,64 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
         d = min(T.alpha, l - unit * T.alpha);
         ntarg = ll - d;
         s0 = src + z * srcz + (size_t)unit * T.alpha * GE::N;
-        gsrc = unit * T.alpha + rank;
+        gsrc = unit * T.alpha + warp;
     } else {
         d = T.alpha;
         ntarg = l;
         s0 = src + z * srcz + ((size_t)unit * ll + l) * GE::N;
-        gsrc = T.L + rank;
-    }
-    const u32 t0 = min(rank * tpc, ntarg), t1 = min(t0 + tpc, ntarg);
-    // constant tables first (overlaps the predecessor's tail)
-    if (rank < d)
-        for (int i = threadIdx.x; i < GE::R / 2; i += blockDim.x)
-            cp_async16(twi + 2 * i, T.colI + (size_t)gsrc * GE::R + 2 * i);
-    for (u32 ti = t0 + grp; ti < t1; ti += NG) {
-        u32 g = ti;
-        if (mode == 0) {
-            const u32 lo = unit * T.alpha;
-            g = glob_of(T, l, ti < lo ? ti : ti + d);
-        }
-        for (int i = tid; i < GE::R / 2; i += GE::COL_THREADS)
-            cp_async16(twt + (size_t)(ti - t0) * GE::R + 2 * i, T.colF + (size_t)g * GE::R + 2 * i);
+        gsrc = T.L + warp;
     }
     pdl_wait();
     pdl_trigger();
-    // phase 1: inverse column pass of this CTA's source limb (group 0), times its scale
-    cp_async_wait_all();
-    __syncthreads();
-    if (rank < d && grp == 0) {
+    if ((u32)warp < d) {
         const u32 q = T.pk[gsrc].q;
         u32 v[16];
-        const u32 *sp = s0 + (size_t)rank * GE::N + col0 + c;
+        gload<PLAST>(v, s0 + (size_t)warp * GE::N + (size_t)col * GE::R, lt);
+        line_inv<GE::LOGR>(v, xl, lt, RowAddr{}, TwRowG{T.colI + (size_t)gsrc * GE::R}, q, SyncWarp{});
+        const uint2 sc = mode == 0 ? T.upScale[(size_t)(d - 1) * T.L + gsrc] : T.downScale[warp];
+        u32 *yt = sy + (warp * GE::CPW + c) * GE::COL_LS;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) v[r] = sp[(size_t)PLAST::x_of(lt, r) * GE::C];
-        line_inv<GE::LOGR>(v, sx, lt, ColAddr<GE::W>{c}, TwNatural{twi}, q, SyncGroup{1, GE::COL_THREADS});
-        const uint2 sc = mode == 0 ? T.upScale[(size_t)(d - 1) * T.L + gsrc] : T.downScale[rank];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) own[PF::x_of(lt, r) * GE::W + c] = shoup(v[r], sc.x, sc.y, q);
-    }
-    cp_async_wait_all();
-    cluster.sync();
-    // phase 2: gather every y tile of the cluster over distributed shared memory
-    for (u32 k = 0; k < d; ++k) {
-        const uint4 *rp = reinterpret_cast<const uint4 *>(cluster.map_shared_rank(own, k));
-        uint4 *lp = reinterpret_cast<uint4 *>(sy + (size_t)k * TILE);
-        for (int e = threadIdx.x; e < TILE / 4; e += blockDim.x) lp[e] = rp[e];
+        for (int r = 0; r < 16; ++r) {
+            const int x = PF::x_of(lt, r);
+            yt[x + (x >> 4)] = shoup(v[r], sc.x, sc.y, q);
+        }
     }
     __syncthreads();
-    // phase 3: this CTA's targets, NG at a time
-    switch (d) {  // uniform over the cluster
-        case 1: colconv_targets<LOGN, 1>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        case 2: colconv_targets<LOGN, 2>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        case 3: colconv_targets<LOGN, 3>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        case 4: colconv_targets<LOGN, 4>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        case 5: colconv_targets<LOGN, 5>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        case 6: colconv_targets<LOGN, 6>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        case 7: colconv_targets<LOGN, 7>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
-        default: colconv_targets<LOGN, 8>(T, mode, out, outz, l, unit, z, t0, t1, sy, sx, twt, grp, NG); break;
+    switch (d) {  // uniform over the CTA
+        case 1: colconv_targets<LOGN, 1, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 2: colconv_targets<LOGN, 2, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 3: colconv_targets<LOGN, 3, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 4: colconv_targets<LOGN, 4, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 5: colconv_targets<LOGN, 5, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 6: colconv_targets<LOGN, 6, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 7: colconv_targets<LOGN, 7, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        default: colconv_targets<LOGN, 8, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
     }
-    cluster.sync();  // no CTA leaves while another may still read its tile
 }
 
 // ------------------------------------------------------------- inner product
-// grid (ROW_BLOCKS, l+alpha, Z).  For target limb t, sum over digits j of
+// grid (ROW_BLOCKS, nt, Z), target limb t = t0 + blockIdx.y.  Sum over digits j of
 // ext_j[t] * (b, a)_{j,g(t)}.  FUSED: ext_j[t] = forward row pass of the
-// column-pass output src[j][t] (or c1[t] for t in D_j); else ext = src.
+// column-major column-pass output src[j][t] (or c1[t] for t in D_j), staged
+// through shared memory one digit ahead; else ext = src (row-major).
 // REGEN: a from ChaCha12 (spec v1), else from the stored key.
-// PINTT: special-prime limbs get the inverse row pass before the store.
+// PINTT: special-prime limbs get the inverse row pass and are stored
+// column-major (the ModDown column kernel reads them so).
 template <int LOGN, bool FUSED, bool REGEN>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 8)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 4)
 k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz,
-        u32 l, KeyPack kp, int pintt) {
+        u32 l, KeyPack kp, int pintt, u32 t0) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
     using PLAST = typename LastPhase<GE::LOGC>::type;
     extern __shared__ __align__(16) u32 dyn[];
-    uint2 *stw = reinterpret_cast<uint2 *>(dyn);          // [NL][C] row twiddles
+    uint2 *stw = reinterpret_cast<uint2 *>(dyn);           // [NL][C] row twiddles
     u32 *sm = dyn + 2 * GE::NL * GE::C;                      // [NL][ROW_LS] exchange
+    u32 *tiles = sm + GE::NL * GE::ROW_LS;                   // [2][C*8] staging
     const int rho = threadIdx.x / GE::TPR, lt = threadIdx.x % GE::TPR;
     const int row0 = blockIdx.x * GE::NL, row = row0 + rho;
-    const u32 t = blockIdx.y, z = blockIdx.z;
+    const u32 t = t0 + blockIdx.y, z = blockIdx.z;
     const u32 ll = l + T.alpha, beta = (l + T.alpha - 1) / T.alpha;
     const u32 g = glob_of(T, l, t);
     const PrimeK pk = T.pk[g];
@@ -378,9 +418,14 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
     const size_t rowoff = (size_t)row * GE::C;
     u32 *line = sm + rho * GE::ROW_LS;
     const TwRow tw{stw + rho * GE::C};
+    const u32 jown = t < l ? t / T.alpha : beta;  // the digit holding t, if any
     if (FUSED) stage_row_tw<GE>(stw, T.rowF + (size_t)g * GE::N + (size_t)row0 * GE::C);
     pdl_wait();
     pdl_trigger();
+    const u32 *srcz_p = src + z * srcz;
+    u32 jn = (jown == 0) ? 1 : 0;  // next converted digit to stage
+    int buf = 0;
+    if (FUSED && jn < beta) stage_cm_rows<GE>(tiles, srcz_p + ((size_t)jn * ll + t) * GE::N, row0);
     u32 seed[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) seed[i] = kp.seed[z][i];
@@ -391,19 +436,30 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
     u64 sb[16], sa[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) { sb[r] = 0; sa[r] = 0; }
-    bool tw_ready = !FUSED;  // uniform over the CTA
 
     for (u32 j = 0; j < beta; ++j) {
-        const bool own = (t < l) && (t / T.alpha == j);
-        // 1. issue this digit's global loads
+        const bool own = j == jown;
         u32 v[16], bv[16], av[16];
-        if (FUSED && !own) gload<PF>(v, src + z * srcz + ((size_t)j * ll + t) * GE::N + rowoff, lt);
-        else if (FUSED) gload<PLAST>(v, c1 + z * c1z + (size_t)t * GE::N + rowoff, lt);
-        else gload<PLAST>(v, src + z * srcz + ((size_t)j * ll + t) * GE::N + rowoff, lt);
+        if (FUSED && !own) {
+            // this digit's tile has landed for every thread; the other tile's
+            // readers (previous converted digit) are done: prefetch the next
+            cp_async_wait_all();
+            __syncthreads();
+            jn = j + 1 + ((j + 1) == jown ? 1 : 0);
+            if (jn < beta) stage_cm_rows<GE>(tiles + (buf ^ 1) * GE::C * 8, srcz_p + ((size_t)jn * ll + t) * GE::N, row0);
+            const u32 *tl = tiles + buf * GE::C * 8;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) v[r] = tl[cm_addr(PF::x_of(lt, r), rho)];
+            buf ^= 1;
+        } else if (FUSED) {
+            gload<PLAST>(v, c1 + z * c1z + (size_t)t * GE::N + rowoff, lt);
+        } else {
+            gload<PLAST>(v, srcz_p + ((size_t)j * ll + t) * GE::N + rowoff, lt);
+        }
         gload<PLAST>(bv, kb + (size_t)j * LLN + (size_t)g * GE::N + rowoff, lt);
         if constexpr (!REGEN) gload<PLAST>(av, ka + (size_t)j * LLN + (size_t)g * GE::N + rowoff, lt);
-        // 2. regenerate a_{j,g} (pure ALU work, overlaps the loads above):
-        //    the thread's elements form groups of KK consecutive coefficients
+        // regenerate a_{j,g} (pure ALU work, overlaps the loads above): the
+        // thread's elements form groups of KK consecutive coefficients
         if constexpr (REGEN) {
 #pragma unroll
             for (int gi = 0; gi < PLAST::G; ++gi) {
@@ -422,16 +478,8 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
                 }
             }
         }
-        // 3. finish the NTT of the converted limb (forward row pass)
-        if (FUSED && !own) {
-            if (!tw_ready) {
-                cp_async_wait_all();
-                __syncthreads();
-                tw_ready = true;
-            }
-            line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
-        }
-        // 4. multiply-accumulate; fold the 64-bit sums every two digits
+        if (FUSED && !own) line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
+        // multiply-accumulate; fold the 64-bit sums every two digits
         const bool fold = (j & 1) && (j + 1 < beta);
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
@@ -452,27 +500,35 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
         ob[r] = shoup(redc64(sb[r], q, pk.qn, pk.q1s), pk.r32, pk.r32s, q);
         oa[r] = shoup(redc64(sa[r], q, pk.qn, pk.q1s), ca, cas, q);
     }
-    u32 *d0 = acc + z * accz + (size_t)t * GE::N + rowoff;
-    u32 *d1 = acc + z * accz + (size_t)(ll + t) * GE::N + rowoff;
+    u32 *d0 = acc + z * accz + (size_t)t * GE::N;
+    u32 *d1 = acc + z * accz + (size_t)(ll + t) * GE::N;
     if (pintt && t >= l) {
         cp_async_wait_all();
-        __syncthreads();  // every reader of the forward table is done
+        __syncthreads();  // every reader of the forward table and the tiles is done
         stage_row_tw<GE>(stw, T.rowI + (size_t)g * GE::N + (size_t)row0 * GE::C);
         cp_async_wait_all();
         __syncthreads();
         line_inv<GE::LOGC>(ob, line, lt, RowAddr{}, tw, q, SyncWarp{});
-        gstore<PF>(ob, d0, lt);
         line_inv<GE::LOGC>(oa, line, lt, RowAddr{}, tw, q, SyncWarp{});
-        gstore<PF>(oa, d1, lt);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int a = cm_addr(PF::x_of(lt, r), rho);
+            tiles[a] = ob[r];
+            tiles[GE::C * 8 + a] = oa[r];
+        }
+        __syncthreads();
+        store_cm_rows<GE>(tiles, d0, row0);
+        store_cm_rows<GE>(tiles + GE::C * 8, d1, row0);
     } else {
-        gstore<PLAST>(ob, d0, lt);
-        gstore<PLAST>(oa, d1, lt);
+        gstore<PLAST>(ob, d0 + rowoff, lt);
+        gstore<PLAST>(oa, d1 + rowoff, lt);
     }
 }
 
 // ----------------------------------------------------------- ModDown finish
 // grid (ROW_BLOCKS, l, Z).  out_h[i] = (acc_h[i] - rowfwd(U_h[i])) [P^-1]_{q_i},
-// plus c0 for h = 0 when c0 is given.  out0/out1 may alias c0 / the input.
+// plus c0 for h = 0 when c0 is given; U column-major, the rest row-major.
+// out0/out1 may alias c0 / the input.
 template <int LOGN>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
@@ -484,6 +540,7 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
     extern __shared__ __align__(16) u32 dyn[];
     uint2 *stw = reinterpret_cast<uint2 *>(dyn);
     u32 *sm = dyn + 2 * GE::NL * GE::C;
+    u32 *tiles = sm + GE::NL * GE::ROW_LS;
     const int rho = threadIdx.x / GE::TPR, lt = threadIdx.x % GE::TPR;
     const int row0 = blockIdx.x * GE::NL, row = row0 + rho;
     const u32 i = blockIdx.y, z = blockIdx.z;
@@ -497,14 +554,16 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
     stage_row_tw<GE>(stw, T.rowF + (size_t)i * GE::N + (size_t)row0 * GE::C);
     pdl_wait();
     pdl_trigger();
-    u32 v0[16], v1[16];
-    gload<PF>(v0, U + z * Uz + (size_t)i * GE::N + rowoff, lt);
-    gload<PF>(v1, U + z * Uz + ((size_t)l + i) * GE::N + rowoff, lt);
+    stage_cm_rows<GE>(tiles, U + z * Uz + (size_t)i * GE::N, row0);
+    stage_cm_rows<GE>(tiles + GE::C * 8, U + z * Uz + ((size_t)l + i) * GE::N, row0);
     cp_async_wait_all();
     __syncthreads();
-    auto half = [&](u32(&v)[16], const int h) {
-        u32 a[16];
+    auto half = [&](const int h) {
+        u32 v[16], a[16];
         gload<PLAST>(a, acc + z * accz + ((size_t)h * ll + i) * GE::N + rowoff, lt);
+        const u32 *tl = tiles + h * GE::C * 8;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) v[r] = tl[cm_addr(PF::x_of(lt, r), rho)];
         line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
         u32 o[16];
 #pragma unroll
@@ -517,8 +576,8 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
         }
         gstore<PLAST>(o, (h == 0 ? out0 : out1) + z * outz + (size_t)i * GE::N + rowoff, lt);
     };
-    half(v0, 0);
-    half(v1, 1);
+    half(0);
+    half(1);
 }
 
 // ------------------------------------------------------------ ModUp finish
@@ -648,23 +707,10 @@ static cudaError_t launch_ex(const pc_ctx *c, void (*kern)(KArgs...), dim3 grid,
     return launch_exc(c, 1, kern, grid, block, smem, s, args...);
 }
 
-// targets per CTA of k_colconv, concurrent target groups, dynamic shared memory
-static u32 colconv_tpc(const pc_ctx *c, int mode, u32 l) {
-    const u32 ntarg_max = mode == 0 ? l + c->alpha - 1 : l;
-    return (ntarg_max + c->alpha - 1) / c->alpha;
-}
-template <int LG>
-static u32 colconv_groups(u32 tpc) {
-    using GE = Geo<LG>;
-    const u32 maxg = 1024 / GE::COL_THREADS;
-    const u32 g = tpc < 4 ? tpc : 4;
-    return g < maxg ? (g ? g : 1) : maxg;
-}
-template <int LG>
-static size_t colconv_smem(const pc_ctx *c, u32 tpc) {
-    using GE = Geo<LG>;
-    return sizeof(u32) * ((size_t)(1 + c->alpha) * GE::R * GE::W + (size_t)colconv_groups<LG>(tpc) * GE::COL_TILE) +
-           sizeof(uint2) * (size_t)(1 + tpc) * GE::R;
+// shared memory of k_colconv: alpha y tiles and two exchange lines per warp
+template <class GE>
+static size_t colconv_smem(const pc_ctx *c) {
+    return sizeof(u32) * (size_t)3 * c->alpha * GE::CPW * GE::COL_LS;
 }
 
 template <class F>
@@ -675,84 +721,108 @@ static cudaError_t allow_smem(F *f, size_t bytes) {
 cudaError_t prepare_kernels(const pc_ctx *c) {
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
-        const size_t rs = row_smem_bytes<GE>();
-        cudaError_t e = allow_smem(k_row<LG, true>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_row<LG, false>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, false>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, true>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, false>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG>, rs);
-        if (e == cudaSuccess) e = allow_smem(k_modup_finish<LG>, rs);
-        // the largest k_colconv instance: ModUp at the top level
-        if (e == cudaSuccess) e = allow_smem(k_colconv<LG>, colconv_smem<LG>(c, colconv_tpc(c, 0, c->L)));
+        cudaError_t e = allow_smem(k_row<LG, true, false>, row_smem_bytes<GE>(0));
+        if (e == cudaSuccess) e = allow_smem(k_row<LG, false, false>, row_smem_bytes<GE>(0));
+        if (e == cudaSuccess) e = allow_smem(k_row<LG, false, true>, row_smem_bytes<GE>(1));
+        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, false>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, true>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, false>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_modup_finish<LG>, row_smem_bytes<GE>(0));
+        if (e == cudaSuccess) e = allow_smem(k_colconv<LG, true>, colconv_smem<GE>(c));
+        if (e == cudaSuccess) e = allow_smem(k_colconv<LG, false>, colconv_smem<GE>(c));
         if (e != cudaSuccess) return e;
     });
     return cudaSuccess;
 }
 
-cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
-                       u32 nlimbs, u32 Z, size_t zin, size_t zout, bool canonical, cudaStream_t s) {
+cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
+                       size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, nlimbs, Z);
-        if (fwd) e = launch_ex(c, k_row<LG, true>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, in, out, first_prime, zin, zout, canonical);
-        else e = launch_ex(c, k_row<LG, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, in, out, first_prime, zin, zout, canonical);
+        if (fwd)
+            e = launch_ex(c, k_row<LG, true, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab,
+                          in, out, first_prime, zin, zout, (int)canonical);
+        else if (cm_out)
+            e = launch_ex(c, k_row<LG, false, true>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(1), s, c->tab,
+                          in, out, first_prime, zin, zout, (int)canonical);
+        else
+            e = launch_ex(c, k_row<LG, false, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab,
+                          in, out, first_prime, zin, zout, (int)canonical);
     });
     return e;
 }
 
-cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
-                       u32 nlimbs, u32 Z, size_t zin, size_t zout, int scale_mode, u32 l,
-                       cudaStream_t s) {
+cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
+                       size_t zin, size_t zout, int scale_mode, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::COL_BLOCKS, nlimbs, Z);
-        if (fwd) e = launch_ex(c, k_col<LG, true>, grid, dim3(GE::COL_THREADS), 0, s, c->tab, in, out, first_prime, zin, zout, scale_mode, l);
-        else e = launch_ex(c, k_col<LG, false>, grid, dim3(GE::COL_THREADS), 0, s, c->tab, in, out, first_prime, zin, zout, scale_mode, l);
+        if (fwd)
+            e = launch_ex(c, k_col<LG, true>, grid, dim3(GE::COL_THREADS), 0, s, c->tab, in, out, first_prime, zin,
+                          zout, scale_mode);
+        else
+            e = launch_ex(c, k_col<LG, false>, grid, dim3(GE::COL_THREADS), 0, s, c->tab, in, out, first_prime, zin,
+                          zout, scale_mode);
     });
     return e;
 }
 
-cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz,
-                           u32 l, u32 Z, cudaStream_t s) {
+cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l,
+                           u32 Z, bool out_cm, cudaStream_t s) {
     const u32 units = mode == 0 ? (l + c->alpha - 1) / c->alpha : 2;
-    const u32 tpc = colconv_tpc(c, mode, l);
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
-        dim3 grid(c->alpha * GE::COL_BLOCKS, 1, units * Z);
-        e = launch_exc(c, c->alpha, k_colconv<LG>, grid, dim3(GE::COL_THREADS * colconv_groups<LG>(tpc)),
-                       colconv_smem<LG>(c, tpc), s, c->tab, mode, src, srcz, out, outz, l, tpc);
+        dim3 grid(GE::C / GE::CPW, 1, units * Z);
+        if (out_cm)
+            e = launch_ex(c, k_colconv<LG, true>, grid, dim3(32 * c->alpha), colconv_smem<GE>(c), s, c->tab, mode,
+                          src, srcz, out, outz, l);
+        else
+            e = launch_ex(c, k_colconv<LG, false>, grid, dim3(32 * c->alpha), colconv_smem<GE>(c), s, c->tab, mode,
+                          src, srcz, out, outz, l);
     });
     return e;
 }
 
-cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz,
-                         const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l, const KeyPack &kp,
-                         u32 Z, bool regen, bool pintt, cudaStream_t s) {
+cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
+                         u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
+                         cudaStream_t s, u32 t0, u32 nt) {
     cudaError_t e = cudaSuccess;
+    if (nt == 0) nt = l + c->alpha - t0;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
-        dim3 grid(GE::ROW_BLOCKS, l + c->alpha, Z);
-        if (fused && regen) e = launch_ex(c, k_inner<LG, true, true>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, src, srcz, c1, c1z, acc, accz, l, kp, pintt);
-        else if (fused) e = launch_ex(c, k_inner<LG, true, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, src, srcz, c1, c1z, acc, accz, l, kp, pintt);
-        else if (regen) e = launch_ex(c, k_inner<LG, false, true>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, src, srcz, c1, c1z, acc, accz, l, kp, pintt);
-        else e = launch_ex(c, k_inner<LG, false, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, src, srcz, c1, c1z, acc, accz, l, kp, pintt);
+        dim3 grid(GE::ROW_BLOCKS, nt, Z);
+        const size_t sm = row_smem_bytes<GE>(2);
+        const int pi = pintt ? 1 : 0;
+        if (fused && regen)
+            e = launch_ex(c, k_inner<LG, true, true>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z,
+                          acc, accz, l, kp, pi, t0);
+        else if (fused)
+            e = launch_ex(c, k_inner<LG, true, false>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z,
+                          acc, accz, l, kp, pi, t0);
+        else if (regen)
+            e = launch_ex(c, k_inner<LG, false, true>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1,
+                          c1z, acc, accz, l, kp, pi, t0);
+        else
+            e = launch_ex(c, k_inner<LG, false, false>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1,
+                          c1z, acc, accz, l, kp, pi, t0);
     });
     return e;
 }
 
-cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc,
-                               size_t accz, const u32 *c0, size_t c0z, u32 *out0, u32 *out1,
-                               size_t outz, u32 l, u32 Z, cudaStream_t s) {
+cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
+                               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, l, Z);
-        e = launch_ex(c, k_moddown_row<LG>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, U, Uz, acc, accz, c0, c0z, out0, out1, outz, l);
+        e = launch_ex(c, k_moddown_row<LG>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(2), s, c->tab, U, Uz,
+                      acc, accz, c0, c0z, out0, out1, outz, l);
     });
     return e;
 }
@@ -762,7 +832,8 @@ cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l,
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, l + c->alpha, (l + c->alpha - 1) / c->alpha);
-        e = launch_ex(c, k_modup_finish<LG>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(), s, c->tab, c1, ext, l);
+        e = launch_ex(c, k_modup_finish<LG>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab, c1, ext,
+                      l);
     });
     return e;
 }

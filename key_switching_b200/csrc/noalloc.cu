@@ -64,8 +64,8 @@ extern "C" int pc_modup_noalloc(pc_ctx *c, const uint32_t *c1, uint32_t l, uint3
     int rc = scratch_address(c->device, &w1);
     if (rc == PC_OK) {
         const cudaStream_t s = (cudaStream_t)stream;
-        cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, s);
-        if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, s);
+        cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, true, s);
+        if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, false, s);
         if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
         if (e != cudaSuccess) rc = pc::record_cuda_error(e);
     }

@@ -133,6 +133,23 @@ __device__ __forceinline__ void exchange(u32 v[16], u32 *sm, int lt, const ADDR 
     for (int r = 0; r < 16; ++r) v[r] = sm[addr(PB::x_of(lt, r))];
 }
 
+template <class PA, class PB, class SYNC, class ADDR>
+__device__ __forceinline__ void exchange2(u32 v0[16], u32 v1[16], u32 *sm0, u32 *sm1, int lt, const ADDR &addr,
+                                          const SYNC &sync) {
+    sync();
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        sm0[addr(PA::x_of(lt, r))] = v0[r];
+        sm1[addr(PA::x_of(lt, r))] = v1[r];
+    }
+    sync();
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        v0[r] = sm0[addr(PB::x_of(lt, r))];
+        v1[r] = sm1[addr(PB::x_of(lt, r))];
+    }
+}
+
 // Full forward line transform: registers enter at Plan::fwd_in positions and
 // leave at Plan::fwd_out positions (lazy values in [0, 2q)).
 template <int LOGM, class ADDR, class TW, class SYNC>
@@ -147,6 +164,27 @@ __device__ __forceinline__ void line_fwd(u32 v[16], u32 *sm, int lt, const ADDR 
     if constexpr (PL::NPH >= 3) {
         exchange<typename PL::P1, typename PL::P2>(v, sm, lt, addr, sync);
         PL::P2::fwd(v, lt, tw, q);
+    }
+}
+
+// Two independent forward line transforms advanced together (separate
+// primes, twiddle tables and exchange lines): twice the independent work
+// between the shared barriers.
+template <int LOGM, class ADDR, class TW0, class TW1, class SYNC>
+__device__ __forceinline__ void line_fwd2(u32 v0[16], u32 v1[16], u32 *sm0, u32 *sm1, int lt, const ADDR &addr,
+                                          const TW0 &tw0, const TW1 &tw1, u32 q0, u32 q1, const SYNC &sync) {
+    using PL = Plan<LOGM>;
+    PL::P0::fwd(v0, lt, tw0, q0);
+    PL::P0::fwd(v1, lt, tw1, q1);
+    if constexpr (PL::NPH >= 2) {
+        exchange2<typename PL::P0, typename PL::P1>(v0, v1, sm0, sm1, lt, addr, sync);
+        PL::P1::fwd(v0, lt, tw0, q0);
+        PL::P1::fwd(v1, lt, tw1, q1);
+    }
+    if constexpr (PL::NPH >= 3) {
+        exchange2<typename PL::P1, typename PL::P2>(v0, v1, sm0, sm1, lt, addr, sync);
+        PL::P2::fwd(v0, lt, tw0, q0);
+        PL::P2::fwd(v1, lt, tw1, q1);
     }
 }
 
@@ -174,15 +212,24 @@ struct TwNatural {
         return t[(1 << s) + (hi << u) + b];
     }
 };
-// Row tables as stored on the device: stages s >= 4 (the distance-1 phase,
-// where every thread of a row has its own twiddles) are re-laid as
-// (1 << s) + (b << 4) + hi, so that at fixed b the threads of a row read
-// consecutive entries (no shared-memory bank conflicts); stages s < 4 are
-// shared by the whole row (broadcast) and keep the natural layout.
+// Twiddle tables as stored on the device ("re-laid"): within stage s, with
+// u = s mod 4 and S0 = s - u (the first stage of its radix-16 phase), the
+// natural entry (1 << s) + (hi << u) + b sits at (1 << s) + (b << S0) + hi.
+// At fixed b the threads of one line (consecutive hi) then read consecutive
+// entries: coalesced from global memory, free of shared-memory bank
+// conflicts.  Stages 0..3 keep the natural order (hi = 0 there: the whole
+// line shares those twiddles).
 struct TwRow {
     const uint2 *t;
     __device__ __forceinline__ uint2 operator()(int s, int u, int hi, int b) const {
-        return s < 4 ? t[(1 << s) + (hi << u) + b] : t[(1 << s) + (b << 4) + hi];
+        return t[(1 << s) + (b << (s - u)) + hi];
+    }
+};
+// The same tables read through the read-only data path.
+struct TwRowG {
+    const uint2 *t;
+    __device__ __forceinline__ uint2 operator()(int s, int u, int hi, int b) const {
+        return __ldg(t + (1 << s) + (b << (s - u)) + hi);
     }
 };
 
@@ -208,21 +255,26 @@ struct Geo {
     static constexpr int LOGC = (LOGN - 4 < 8) ? LOGN - 4 : 8;
     static constexpr int LOGR = LOGN - LOGC;
     static constexpr int N = 1 << LOGN, C = 1 << LOGC, R = 1 << LOGR;
-    // row pass: NL rows per CTA (64 threads), C/16 threads per row
+    // row pass: NL = 8 rows per CTA (a 32-byte segment of every column of a
+    // column-major limb), C/16 threads per row
     static constexpr int TPR = C / 16;
-    static constexpr int NL = (64 / TPR < R) ? 64 / TPR : R;
+    static constexpr int NL = 8;
     static constexpr int ROW_THREADS = NL * TPR;
     static constexpr int ROW_BLOCKS = R / NL;
     static constexpr int ROW_LS = C + C / 16;  // padded row stride in shared memory
-    // column pass: W columns per CTA (128..256 threads), R/16 threads per column;
-    // the shared tile is row-major with one W-word pad every 16 rows, which
-    // keeps the phase exchanges free of bank conflicts
+    // column pass on a row-major limb (the NTT calls): W columns per CTA,
+    // R/16 threads per column, CTA barriers between phases; the shared tile
+    // is row-major with one W-word pad every 16 rows
     static constexpr int TPCOL = R / 16;
     static constexpr int W_ = 2048 / R > 4 ? 2048 / R : 4;
     static constexpr int W = W_ < C ? W_ : C;
     static constexpr int COL_THREADS = W * TPCOL;
     static constexpr int COL_BLOCKS = C / W;
     static constexpr int COL_TILE = (R + R / 16) * W;  // words of the padded tile
+    // column pass on a column-major limb (the key-switch kernels): one column
+    // per TPCOL consecutive lanes, CPW columns per warp, warp barriers only
+    static constexpr int CPW = 32 / TPCOL;
+    static constexpr int COL_LS = R + R / 16;  // padded column stride in shared memory
     static_assert(LOGC >= 4 && LOGR >= 4 && LOGR <= 9, "supported 2^8..2^17 (R,C >= 16)");
 };
 

@@ -68,6 +68,11 @@ struct pc_ctx {
     void *l2_window_base;
     size_t l2_window_bytes;
     float l2_hit_ratio;
+    // internal high-priority stream and fork / join events: the ModDown
+    // branch of a key switch overlaps the ciphertext-prime inner products
+    int overlap;
+    cudaStream_t aux;
+    cudaEvent_t ev_fork, ev_join;
     // per-kernel timing (pc_profile_begin / pc_profile_end)
     cudaEvent_t *prof_ev;   // [prof_max][PC_PROFILE_STAGES + 1]
     uint32_t prof_max, prof_used, prof_every, prof_seen;
@@ -75,27 +80,27 @@ struct pc_ctx {
 
 namespace pc {
 
-// launchers (kernels.cu); each returns a cudaError_t from the launch
-cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
-                       u32 nlimbs, u32 Z, size_t zin, size_t zout, bool canonical, cudaStream_t s);
-// scale_mode: 0 none, 1 N^-1, 2 ModUp digit scale at level l, 3 ModDown P-hat scale
-cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime,
-                       u32 nlimbs, u32 Z, size_t zin, size_t zout, int scale_mode, u32 l,
-                       cudaStream_t s);
-// fused cluster kernel: inverse column pass + scale of the sources, DSMEM
-// gather, conversion and forward column pass of the targets.  mode 0 (ModUp):
-// src = the inverse-row-pass output of c1 [l][N], out = T [beta][l+alpha][N];
-// mode 1 (ModDown): src = ACC [2][l+alpha][N] (special limbs row-inverted),
-// out = U [2][l][N]
-
-cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz,
-                           u32 l, u32 Z, cudaStream_t s);
-cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz,
-                         const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l, const KeyPack &kp,
-                         u32 Z, bool regen, bool pintt, cudaStream_t s);
-cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc,
-                               size_t accz, const u32 *c0, size_t c0z, u32 *out0, u32 *out1,
-                               size_t outz, u32 l, u32 Z, cudaStream_t s);
+// launchers (kernels.cu); each returns a cudaError_t from the launch.
+// "CM" = column-major limb (element (r, c) at c*R + r), used for the
+// intermediates between row passes and column passes.
+cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
+                       size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s);
+// scale_mode: 0 none (lazy), 1 N^-1 (canonical)
+cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
+                       size_t zin, size_t zout, int scale_mode, cudaStream_t s);
+// conversion kernel: inverse column pass + scale of the sources (CM), basis
+// conversion and forward column pass of the targets.  mode 0 (ModUp):
+// src = INTT-row output of c1 (CM) [l][N], out = [beta][l+alpha][N];
+// mode 1 (ModDown): src = ACC [2][l+alpha][N] (special limbs CM),
+// out = [2][l][N].  Output CM when out_cm, else row-major.
+cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l,
+                           u32 Z, bool out_cm, cudaStream_t s);
+// inner product for target limbs t0 .. t0+nt-1 (nt = 0: through l+alpha-1)
+cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
+                         u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
+                         cudaStream_t s, u32 t0 = 0, u32 nt = 0);
+cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
+                               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s);
 cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l, cudaStream_t s);
 cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, cudaStream_t s);
 cudaError_t prepare_kernels(const pc_ctx *c);
