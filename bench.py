@@ -32,6 +32,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 2**20
+# DRAM bytes (read + write) per launch of the roofline kernel, from one ncu
+# capture of the current kernel (profiles/k_inner_keyswitch_n16.md, cold
+# cache); None when the kernel has changed since the counters were taken.
+KERNEL_TRAFFIC = {("rot1_n16", "inner_chacha"): 105.10e6 + 4.92e6}
 MODMUL_IMAD = 3      # IMAD-pipe instructions of one Shoup modular multiply
 IMAD_PER_SM_CLK = 64  # 32-bit IMAD lanes per SM per clock
 SMS = 148
@@ -217,7 +221,9 @@ def run_ours(args):
                     ctx.keyswitch(c0, c1, l, keys[0], out[0, 0, :l], out[0, 1, :l], stream)
                 else:
                     ctx.keyswitch_batch(ct, B, l, keys, out, stream)
-        launches_per_step = 5 * len(levels)
+        # 6 launches per key switch (the inner product splits in two when the
+        # ModDown branch overlaps), 5 in the instrumented (serial) calls
+        launches_per_step = (5 if os.environ.get("PC_NO_OVERLAP") else 6) * len(levels)
         work = [workload_counts(wl.logN, L, A, l, regen) for l in levels]
 
     # warm-up, then exactly K timed steps between barriers
@@ -262,7 +268,8 @@ def run_ours(args):
                       f"{'regenerated in-kernel (ChaCha12)' if regen else 'stored in HBM'}",
                       "l2": f"inputs rotated over {nsets} sets of {per_set / 1e6:.1f} MB (> 126 MB L2)",
                       "parallelism": f"replicas x{world}"},
-           "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+           "gpu_launches": launches_per_step * args.steps
+           - (0 if (os.environ.get("PC_NO_OVERLAP") or not prof) else ncalls), "clocks": clk}
 
     if work is not None:
         mm = sum(w["modmuls"] for w in work)
@@ -295,8 +302,11 @@ def run_ours(args):
             ach = smm[top] / per_launch_s
             res["roofline"] = {"bound": "alu", "kernel": top, "achieved": ach / 1e12,
                                "peak": peak_derived / 1e12, "unit": "Tmodmul/s",
-                               "frac": ach / peak_derived, "traffic": None,
-                               "share": stage_ms[top] / tot if tot else None}
+                               "frac": ach / peak_derived,
+                               "traffic": KERNEL_TRAFFIC.get((args.workload, top)) if regen else None,
+                               "share": stage_ms[top] / tot if tot else None,
+                               "peak_source": "derived: 148 SMs x 64 IMAD lanes/clk x 1965 MHz / 3 IMAD per "
+                                              "Shoup modular multiply"}
             res["stage_ms_per_step"] = {k: v / ncalls * len(levels) for k, v in stage_ms.items()}
             res["stage_sampling"] = f"{ncalls} of {args.steps * len(levels)} calls instrumented (every {PROF_EVERY}th)"
 
