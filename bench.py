@@ -36,7 +36,10 @@ L2_BYTES = 126 * 2**20
 # capture of the current kernel (profiles/k_inner_keyswitch_n16.md, cold
 # cache); None when the kernel has changed since the counters were taken.
 KERNEL_TRAFFIC = {("rot1_n16", "inner_chacha"): 105.10e6 + 4.92e6}
-MODMUL_IMAD = 3      # IMAD-pipe instructions of one Shoup modular multiply
+# A Shoup modular multiply is IMAD.HI + 2 IMAD on the 16-lane-per-partition
+# multiply-add pipe, and the high-half multiply occupies two issue slots:
+# 4 slots of 64 lanes/SM/clock (measured by pc_microbench kind 0 at 4.57 T/s)
+MODMUL_IMAD = 4
 IMAD_PER_SM_CLK = 64  # 32-bit IMAD lanes per SM per clock
 SMS = 148
 
@@ -305,8 +308,8 @@ def run_ours(args):
                                "frac": ach / peak_derived,
                                "traffic": KERNEL_TRAFFIC.get((args.workload, top)) if regen else None,
                                "share": stage_ms[top] / tot if tot else None,
-                               "peak_source": "derived: 148 SMs x 64 IMAD lanes/clk x 1965 MHz / 3 IMAD per "
-                                              "Shoup modular multiply"}
+                               "peak_source": "derived: 148 SMs x 64 IMAD lanes/clk x 1965 MHz / 4 multiply-pipe "
+                                              "slots per Shoup modular multiply (IMAD.HI is two)"}
             res["stage_ms_per_step"] = {k: v / ncalls * len(levels) for k, v in stage_ms.items()}
             res["stage_sampling"] = f"{ncalls} of {args.steps * len(levels)} calls instrumented (every {PROF_EVERY}th)"
 

@@ -12,6 +12,7 @@
 //   4: 32-bit add + xor (IADD3 / LOP3)       -> instructions/s
 //   5..8: ChaCha12 blocks with rotation subsets on the multiply pipe
 //         (mask 1: rot16; 5: rot16+rot8; 3: rot16+rot12; 15: all) -> blocks/s
+//   9: ChaCha12, two blocks with interleaved quarter rounds  -> blocks/s
 #include <cuda_runtime.h>
 
 #include "chacha.cuh"
@@ -63,6 +64,13 @@ __global__ void __launch_bounds__(MB_THREADS) k_micro(u32 iters, u32 q, u32 w, u
             chacha12_block(k, it, tid, 0, out);
 #pragma unroll
             for (int i = 0; i < 8; ++i) x[i] ^= out[i] + out[i + 8];
+        } else if constexpr (KIND == 9) {
+            u32 k[8], o0[16], o1[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) k[i] = x[i];
+            chacha12_block2(k, 2 * it, tid, 0, o0, o1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] ^= o0[i] + o1[i + 8];
         } else if constexpr (KIND >= 5) {
             constexpr int MASK = KIND == 5 ? 1 : KIND == 6 ? 5 : KIND == 7 ? 3 : 15;
             const u32 mul[4] = {w & 0 | (1u << 16), 1u << 12, 1u << 8, 1u << 7};
@@ -110,7 +118,7 @@ static cudaError_t run_micro(int sms, u32 iters, u32 *sink, float *ms) {
 
 extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s) {
     using namespace pc;
-    if (!ops_per_s || kind < 0 || kind > 8 || iters < 1) return PC_E_ARG;
+    if (!ops_per_s || kind < 0 || kind > 9 || iters < 1) return PC_E_ARG;
     if (cudaSetDevice(device) != cudaSuccess) return PC_E_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return PC_E_CUDA;
@@ -127,12 +135,13 @@ extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_p
         case 6: e = run_micro<6>(sms, iters, sink, &ms); break;
         case 7: e = run_micro<7>(sms, iters, sink, &ms); break;
         case 8: e = run_micro<8>(sms, iters, sink, &ms); break;
+        case 9: e = run_micro<9>(sms, iters, sink, &ms); break;
         default: e = run_micro<4>(sms, iters, sink, &ms); break;
     }
     cudaFree(sink);
     if (e != cudaSuccess || ms <= 0.f) return PC_E_CUDA;
     const double threads = (double)sms * 8 * MB_THREADS;
-    const double per_iter = (kind == 2 || kind >= 5) ? 1.0 : (double)MB_CHAINS;
+    const double per_iter = kind == 9 ? 2.0 : (kind == 2 || kind >= 5) ? 1.0 : (double)MB_CHAINS;
     *ops_per_s = threads * per_iter * (double)iters / (ms * 1e-3);
     return PC_OK;
 }
