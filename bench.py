@@ -147,6 +147,24 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The largest value of x over all ranks (every rank gets it); x itself
+    without a process group.  Used for the device-timed region, so the
+    slowest rank sets the job's time."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank processes its own units
+    (weak scaling), the time is the slowest rank's."""
+    return units_per_rank_step * steps * world / (max_ms * 1e-3)
+
+
 # --------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -255,12 +273,8 @@ def run_ours(args):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     stage_ms, ncalls = ctx.profile_end() if prof else ({}, 0)
-    if dist:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    total_units = units_per_step * args.steps * world
-    value = total_units / (ms * 1e-3)
+    ms = max_over_ranks(ms, dist, "cuda")
+    value = whole_job_rate(units_per_step, args.steps, world, ms)
 
     res = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -338,11 +352,8 @@ def run_ours(args):
         f1.record(stream)
         torch.cuda.synchronize()
         ems = f0.elapsed_time(f1)
-        if dist:
-            t = torch.tensor([ems], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        res["e2e"] = {"value": ke * world / (ems * 1e-3), "unit": unit,
+        ems = max_over_ranks(ems, dist, "cuda")
+        res["e2e"] = {"value": whole_job_rate(1, ke, world, ems), "unit": unit,
                       "h2d_bytes_per_step": 2 * l * N * 4, "d2h_bytes_per_step": 2 * l * N * 4}
 
     if rank == 0 and not args.no_cpu_baseline and args.workload in ("rot1_n16", "relin_n12"):
