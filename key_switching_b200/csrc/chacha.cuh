@@ -33,6 +33,16 @@ struct ChaRot {
     }
 };
 
+// Byte-aligned rotations (16 and 8) as byte permutes, the others as funnel
+// shifts.
+struct ChaRotPrmt {
+    __device__ __forceinline__ uint32_t r(int i, uint32_t x) const {
+        if (i == 0) return __byte_perm(x, x, 0x1032);
+        if (i == 2) return __byte_perm(x, x, 0x2103);
+        return rotl32(x, i == 1 ? 12 : 7);
+    }
+};
+
 #define PC_QR(a, b, c, d)                          \
     a += b; d ^= a; d = R.r(0, d);                 \
     c += d; b ^= c; b = R.r(1, b);                 \
@@ -40,9 +50,9 @@ struct ChaRot {
     c += d; b ^= c; b = R.r(3, b);
 
 // out[16] = ChaCha12(seed words k[8], counter, g, j)
-template <int MULMASK = 0>
+template <class ROT = ChaRot<0>>
 __device__ __forceinline__ void chacha12_block(const uint32_t k[8], uint32_t ctr, uint32_t g, uint32_t j,
-                                               uint32_t out[16], const ChaRot<MULMASK> &R = ChaRot<MULMASK>{}) {
+                                               uint32_t out[16], const ROT &R = ROT{}) {
     const uint32_t c0 = 0x61707865u, c1 = 0x3320646eu, c2 = 0x79622d32u, c3 = 0x6b206574u;
     uint32_t x0 = c0, x1 = c1, x2 = c2, x3 = c3;
     uint32_t x4 = k[0], x5 = k[1], x6 = k[2], x7 = k[3];

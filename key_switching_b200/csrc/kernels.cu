@@ -34,6 +34,13 @@
 
 namespace pc {
 
+// Minimum resident CTAs per SM given to __launch_bounds__.  Without one,
+// ptxas fits the kernels into 32 registers (full occupancy); these
+// latency-bound kernels run faster with the registers they naturally use
+// (48-105), which keep more independent loads and butterflies in flight.
+constexpr int ROW_MIN_CTAS = 8;
+constexpr int COLCONV_MIN_CTAS = 1;
+
 // ------------------------------------------------------------------ helpers
 
 // global prime index of local limb t at level l
@@ -144,7 +151,7 @@ constexpr size_t row_smem_bytes(int tiles) {
 // grid (ROW_BLOCKS, nlimbs, Z).  Row-major limbs in.  Out: row-major (in
 // place allowed), or for CMOUT (inverse only) column-major limbs.
 template <int LOGN, bool FWD, bool CMOUT>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int canonical) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
@@ -194,7 +201,7 @@ k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
 // (the NTT calls).  grid (COL_BLOCKS, nlimbs, Z).  In place allowed.
 // scale_mode 0: lazy output; 1: times N^-1, canonical.
 template <int LOGN, bool FWD>
-__global__ void __launch_bounds__(Geo<LOGN>::COL_THREADS)
+__global__ void __launch_bounds__(Geo<LOGN>::COL_THREADS, ROW_MIN_CTAS)
 k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int scale_mode) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
@@ -250,7 +257,7 @@ k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
 // false).  grid (C / CPW, 1, units * Z), block 32 * alpha.
 template <int LOGN, int D, bool OUT_CM>
 __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *out, size_t outz, u32 l, u32 unit,
-                                                u32 z, u32 ntarg, const u32 *sy, u32 *xl0, u32 *xl1, int c, int lt,
+                                                u32 z, u32 ntarg, const u32 *sy, u32 *xl0, int c, int lt,
                                                 int col) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
@@ -272,65 +279,43 @@ __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *
             dst = out + z * outz + ((size_t)unit * l + ti) * GE::N;
         }
     };
-    // two targets per warp at a time: ti and ti + nwarps
-    for (u32 ti = warp; ti < ntarg; ti += 2 * nwarps) {
-        const u32 tj = ti + nwarps;
-        const bool two = tj < ntarg;
-        u32 g0, g1;
-        const u32 *conv0, *conv1;
-        u32 *dst0, *dst1;
+    // one target per warp at a time (a short loop body: the kernel is
+    // latency-bound and a two-target body overflowed the instruction cache)
+    for (u32 ti = warp; ti < ntarg; ti += nwarps) {
+        u32 g0;
+        const u32 *conv0;
+        u32 *dst0;
         target(ti, g0, conv0, dst0);
-        target(two ? tj : ti, g1, conv1, dst1);
         const u32 q0 = T.pk[g0].q, qn0 = T.pk[g0].qn, q1s0 = T.pk[g0].q1s;
-        const u32 q1 = T.pk[g1].q, qn1 = T.pk[g1].qn, q1s1 = T.pk[g1].q1s;
-        u32 cv0[D], cv1[D];
+        u32 cv0[D];
 #pragma unroll
-        for (int k = 0; k < D; ++k) {
-            cv0[k] = __ldg(conv0 + k);
-            cv1[k] = __ldg(conv1 + k);
-        }
-        u32 v0[16], v1[16];
+        for (int k = 0; k < D; ++k) cv0[k] = __ldg(conv0 + k);
+        u32 v0[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const int x = PF::x_of(lt, r);
             const int xa = c * GE::COL_LS + x + (x >> 4);
-            u64 a0 = 0, a1 = 0;
+            u64 a0 = 0;
 #pragma unroll
             for (int k = 0; k < D; ++k) {
-                if (k == 4 || k == 6) {
-                    a0 = fold64(a0, q0, q1s0);
-                    a1 = fold64(a1, q1, q1s1);
-                }
-                const u32 y = sy[k * GE::CPW * GE::COL_LS + xa];
-                a0 += (u64)y * cv0[k];
-                a1 += (u64)y * cv1[k];
+                if (k == 4 || k == 6) a0 = fold64(a0, q0, q1s0);
+                a0 += (u64)sy[k * GE::CPW * GE::COL_LS + xa] * cv0[k];
             }
-            if constexpr (D <= 4) {
-                v0[r] = redc((u32)a0, red1((u32)(a0 >> 32), q0), q0, qn0);
-                v1[r] = redc((u32)a1, red1((u32)(a1 >> 32), q1), q1, qn1);
-            } else {
-                v0[r] = redc64(a0, q0, qn0, q1s0);
-                v1[r] = redc64(a1, q1, qn1, q1s1);
-            }
+            if constexpr (D <= 4) v0[r] = redc((u32)a0, red1((u32)(a0 >> 32), q0), q0, qn0);
+            else v0[r] = redc64(a0, q0, qn0, q1s0);
         }
-        line_fwd2<GE::LOGR>(v0, v1, xl0, xl1, lt, RowAddr{}, TwRowG{T.colF + (size_t)g0 * GE::R},
-                            TwRowG{T.colF + (size_t)g1 * GE::R}, q0, q1, SyncWarp{});
+        line_fwd<GE::LOGR>(v0, xl0, lt, RowAddr{}, TwRowG{T.colF + (size_t)g0 * GE::R}, q0, SyncWarp{});
         if constexpr (OUT_CM) {
             gstore<PLAST>(v0, dst0 + (size_t)col * GE::R, lt);
-            if (two) gstore<PLAST>(v1, dst1 + (size_t)col * GE::R, lt);
         } else {
 #pragma unroll
             for (int r = 0; r < 16; ++r) dst0[(size_t)PLAST::x_of(lt, r) * GE::C + col] = v0[r];
-            if (two) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r) dst1[(size_t)PLAST::x_of(lt, r) * GE::C + col] = v1[r];
-            }
         }
     }
 }
 
 template <int LOGN, bool OUT_CM>
-__global__ void __launch_bounds__(32 * MAX_ALPHA)
+__global__ void __launch_bounds__(32 * MAX_ALPHA, COLCONV_MIN_CTAS)
 k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
@@ -341,9 +326,8 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
     const int c = lane / GE::TPCOL, lt = lane % GE::TPCOL;
     const int col = blockIdx.x * GE::CPW + c;
     u32 *sy = dyn;                                          // [alpha][CPW][COL_LS] y tiles
-    // two exchange lines per warp and column
-    u32 *xl = dyn + (T.alpha + 2 * warp) * GE::CPW * GE::COL_LS + c * GE::COL_LS;
-    u32 *xl1 = xl + GE::CPW * GE::COL_LS;
+    // one exchange line per warp and column
+    u32 *xl = dyn + (T.alpha + warp) * GE::CPW * GE::COL_LS + c * GE::COL_LS;
     const u32 units = mode == 0 ? (l + T.alpha - 1) / T.alpha : 2;
     const u32 z = blockIdx.z / units, unit = blockIdx.z % units;
     const u32 ll = l + T.alpha;
@@ -377,14 +361,14 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
     }
     __syncthreads();
     switch (d) {  // uniform over the CTA
-        case 1: colconv_targets<LOGN, 1, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        case 2: colconv_targets<LOGN, 2, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        case 3: colconv_targets<LOGN, 3, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        case 4: colconv_targets<LOGN, 4, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        case 5: colconv_targets<LOGN, 5, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        case 6: colconv_targets<LOGN, 6, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        case 7: colconv_targets<LOGN, 7, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
-        default: colconv_targets<LOGN, 8, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, xl1, c, lt, col); break;
+        case 1: colconv_targets<LOGN, 1, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 2: colconv_targets<LOGN, 2, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 3: colconv_targets<LOGN, 3, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 4: colconv_targets<LOGN, 4, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 5: colconv_targets<LOGN, 5, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 6: colconv_targets<LOGN, 6, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 7: colconv_targets<LOGN, 7, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        default: colconv_targets<LOGN, 8, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
     }
 }
 
@@ -530,7 +514,7 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
 // plus c0 for h = 0 when c0 is given; U column-major, the rest row-major.
 // out0/out1 may alias c0 / the input.
 template <int LOGN>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l) {
     using GE = Geo<LOGN>;
@@ -584,7 +568,7 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
 // grid (ROW_BLOCKS, l+alpha, beta).  ext[j][t] = c1[t] for t in D_j, else the
 // forward row pass (in place) of the column-pass output already in ext[j][t].
 template <int LOGN>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_modup_finish(Tables T, const u32 *c1, u32 *ext, u32 l) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
@@ -707,10 +691,10 @@ static cudaError_t launch_ex(const pc_ctx *c, void (*kern)(KArgs...), dim3 grid,
     return launch_exc(c, 1, kern, grid, block, smem, s, args...);
 }
 
-// shared memory of k_colconv: alpha y tiles and two exchange lines per warp
+// shared memory of k_colconv: alpha y tiles and one exchange line per warp
 template <class GE>
 static size_t colconv_smem(const pc_ctx *c) {
-    return sizeof(u32) * (size_t)3 * c->alpha * GE::CPW * GE::COL_LS;
+    return sizeof(u32) * (size_t)2 * c->alpha * GE::CPW * GE::COL_LS;
 }
 
 template <class F>

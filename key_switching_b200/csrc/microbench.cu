@@ -13,6 +13,7 @@
 //   5..8: ChaCha12 blocks with rotation subsets on the multiply pipe
 //         (mask 1: rot16; 5: rot16+rot8; 3: rot16+rot12; 15: all) -> blocks/s
 //   9: ChaCha12, two blocks with interleaved quarter rounds  -> blocks/s
+//  10: ChaCha12 with the 16- and 8-bit rotations as byte permutes -> blocks/s
 #include <cuda_runtime.h>
 
 #include "chacha.cuh"
@@ -32,7 +33,7 @@ __device__ __forceinline__ void micro_chacha(u32 x[MB_CHAINS], u32 it, u32 tid, 
     u32 k[8], out[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) k[i] = x[i];
-    chacha12_block<MASK>(k, it, tid, 0, out, R);
+    chacha12_block(k, it, tid, 0, out, R);
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[i] ^= out[i] + out[i + 8];
 }
@@ -62,6 +63,13 @@ __global__ void __launch_bounds__(MB_THREADS) k_micro(u32 iters, u32 q, u32 w, u
 #pragma unroll
             for (int i = 0; i < 8; ++i) k[i] = x[i];
             chacha12_block(k, it, tid, 0, out);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] ^= out[i] + out[i + 8];
+        } else if constexpr (KIND == 10) {
+            u32 k[8], out[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) k[i] = x[i];
+            chacha12_block(k, it, tid, 0, out, ChaRotPrmt{});
 #pragma unroll
             for (int i = 0; i < 8; ++i) x[i] ^= out[i] + out[i + 8];
         } else if constexpr (KIND == 9) {
@@ -118,7 +126,7 @@ static cudaError_t run_micro(int sms, u32 iters, u32 *sink, float *ms) {
 
 extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s) {
     using namespace pc;
-    if (!ops_per_s || kind < 0 || kind > 9 || iters < 1) return PC_E_ARG;
+    if (!ops_per_s || kind < 0 || kind > 10 || iters < 1) return PC_E_ARG;
     if (cudaSetDevice(device) != cudaSuccess) return PC_E_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return PC_E_CUDA;
@@ -136,6 +144,7 @@ extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_p
         case 7: e = run_micro<7>(sms, iters, sink, &ms); break;
         case 8: e = run_micro<8>(sms, iters, sink, &ms); break;
         case 9: e = run_micro<9>(sms, iters, sink, &ms); break;
+        case 10: e = run_micro<10>(sms, iters, sink, &ms); break;
         default: e = run_micro<4>(sms, iters, sink, &ms); break;
     }
     cudaFree(sink);
