@@ -404,6 +404,17 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
     const TwRow tw{stw + rho * GE::C};
     const u32 jown = t < l ? t / T.alpha : beta;  // the digit holding t, if any
     if (FUSED) stage_row_tw<GE>(stw, T.rowF + (size_t)g * GE::N + (size_t)row0 * GE::C);
+    // counter-free quarter rounds of every digit's ChaCha12 blocks, once per CTA
+    __shared__ __align__(16) u32 spre[12 * MAX_L];
+    if (REGEN && threadIdx.x < beta) {
+        u32 sd[8], pre[12];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sd[i] = kp.seed[z][i];
+        chacha12_precolumn(sd, g, threadIdx.x, pre);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) spre[12 * threadIdx.x + i] = pre[i];
+    }
+    __syncthreads();
     pdl_wait();
     pdl_trigger();
     const u32 *srcz_p = src + z * srcz;
@@ -444,7 +455,24 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
         if constexpr (!REGEN) gload<PLAST>(av, ka + (size_t)j * LLN + (size_t)g * GE::N + rowoff, lt);
         // regenerate a_{j,g} (pure ALU work, overlaps the loads above): the
         // thread's elements form groups of KK consecutive coefficients
-        if constexpr (REGEN) {
+        if constexpr (REGEN && PLAST::KK == 16) {
+            // the thread's 16 consecutive coefficients are two whole blocks
+            const u32 base = (u32)(rowoff + PLAST::x_of(lt, 0));
+            u32 o0[16], o1[16];
+            u32 pre[12];
+            const uint4 *pp = reinterpret_cast<const uint4 *>(spre + 12 * j);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const uint4 w4 = pp[i];
+                pre[4 * i] = w4.x; pre[4 * i + 1] = w4.y; pre[4 * i + 2] = w4.z; pre[4 * i + 3] = w4.w;
+            }
+            chacha12_block2_pre(pre, seed, base >> 3, g, j, o0, o1);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                av[w] = redc(o0[2 * w], mod32(o0[2 * w + 1], q, pk.q1s), q, pk.qn);
+                av[8 + w] = redc(o1[2 * w], mod32(o1[2 * w + 1], q, pk.q1s), q, pk.qn);
+            }
+        } else if constexpr (REGEN) {
 #pragma unroll
             for (int gi = 0; gi < PLAST::G; ++gi) {
                 const u32 base = (u32)(rowoff + PLAST::x_of(lt, gi * PLAST::KK));
