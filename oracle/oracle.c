@@ -445,6 +445,131 @@ int or_keyswitch(const or_params *P, const uint32_t *c0, const uint32_t *c1, uin
 }
 
 /* ------------------------------------------------------------------ */
+/* rotations (automorphism X -> X^g followed by a key switch)          */
+/* ------------------------------------------------------------------ */
+/* NTT-domain automorphism: slot k of the forward transform holds
+ * a(psi^(2 brv(k) + 1)), so slot k of NTT(a(X^g)) is a(psi^(g (2 brv(k) + 1))),
+ * the slot k' of NTT(a) with 2 brv(k') + 1 = g (2 brv(k) + 1) mod 2N.
+ * g odd; one limb of N words. */
+void or_automorph_ntt(const uint32_t *in, uint32_t logN, uint32_t g, uint32_t *out) {
+    uint32_t N = 1u << logN;
+    uint64_t twoN = 2ull * N;
+    for (uint32_t k = 0; k < N; k++) {
+        uint64_t e = ((2ull * bitrev(k, logN) + 1) * g) % twoN;
+        uint32_t kp = bitrev((uint32_t)((e - 1) / 2), logN);
+        out[k] = in[kp];
+    }
+}
+
+/* Rotation of (c0, c1) (decrypting under s) by the Galois element g:
+ * (c0(X^g), c1(X^g)) decrypts under s(X^g); key switch it with a key for
+ * s(X^g) -> s.  The automorphism is applied to the input limbs first. */
+int or_rotate(const or_params *P, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t g,
+              const uint8_t seed[32], const uint32_t *b, const uint32_t *a, int rounds,
+              uint32_t *c0o, uint32_t *c1o) {
+    if (check_params(P, l) || (g & 1u) == 0 || g >= (2u << P->logN)) return -1;
+    uint32_t N = 1u << P->logN;
+    uint32_t *r0 = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)l * N);
+    uint32_t *r1 = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)l * N);
+    for (uint32_t i = 0; i < l; i++) {
+        or_automorph_ntt(c0 + (size_t)i * N, P->logN, g, r0 + (size_t)i * N);
+        or_automorph_ntt(c1 + (size_t)i * N, P->logN, g, r1 + (size_t)i * N);
+    }
+    int rc = or_keyswitch(P, r0, r1, l, seed, b, a, rounds, c0o, c1o);
+    free(r1);
+    free(r0);
+    return rc;
+}
+
+/* One rotation of a hoisted batch: ext = ModUp(c1) is computed once for all
+ * rotations of the same ciphertext; this rotation applies the automorphism to
+ * every limb of ext (it commutes with the inner product and ModDown, and a
+ * permuted lift is still a lift of c1(X^g)), then finishes like a key switch
+ * with c0(X^g). */
+int or_rotate_hoisted_one(const or_params *P, const uint32_t *c0, const uint32_t *ext, uint32_t l,
+                          uint32_t g, const uint8_t seed[32], const uint32_t *b, const uint32_t *a,
+                          int rounds, uint32_t *c0o, uint32_t *c1o) {
+    if (check_params(P, l) || (g & 1u) == 0 || g >= (2u << P->logN)) return -1;
+    uint32_t N = 1u << P->logN, al = P->alpha, beta = (l + al - 1) / al, ll = l + al;
+    uint32_t *er = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)beta * ll * N);
+    uint32_t *acc = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)2 * ll * N);
+    uint32_t *out = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)2 * l * N);
+    uint32_t *r0 = (uint32_t *)malloc(sizeof(uint32_t) * N);
+    for (size_t m = 0; m < (size_t)beta * ll; m++) or_automorph_ntt(ext + m * N, P->logN, g, er + m * N);
+    int rc = or_inner(P, er, l, seed, b, a, rounds, acc);
+    if (!rc) rc = or_moddown(P, acc, l, out);
+    if (!rc) {
+        for (uint32_t i = 0; i < l; i++) {
+            uint32_t qi = P->q[i];
+            or_automorph_ntt(c0 + (size_t)i * N, P->logN, g, r0);
+            for (uint32_t n = 0; n < N; n++) {
+                size_t o = (size_t)i * N + n;
+                c0o[o] = addm(r0[n], out[o], qi);
+                c1o[o] = out[(size_t)l * N + o];
+            }
+        }
+    }
+    free(r0);
+    free(out);
+    free(acc);
+    free(er);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* relinearisation (ciphertext product)                                */
+/* ------------------------------------------------------------------ */
+/* Tensor of two ciphertexts (x0, x1), (y0, y1) at level l, NTT domain, where
+ * the ring product is the slot-wise product:
+ *   d0 = x0 y0,  d1 = x0 y1 + x1 y0,  d2 = x1 y1      (d0 + d1 s + d2 s^2)
+ * then d2 is key-switched with a key for s^2 -> s:
+ *   c0' = d0 + ModDown_b,  c1' = d1 + ModDown_a. */
+int or_tensor(const or_params *P, const uint32_t *x0, const uint32_t *x1, const uint32_t *y0,
+              const uint32_t *y1, uint32_t l, uint32_t *d0, uint32_t *d1, uint32_t *d2) {
+    if (check_params(P, l)) return -1;
+    uint32_t N = 1u << P->logN;
+    for (uint32_t i = 0; i < l; i++) {
+        uint32_t q = P->q[i];
+        for (uint32_t n = 0; n < N; n++) {
+            size_t o = (size_t)i * N + n;
+            d0[o] = mulm(x0[o], y0[o], q);
+            d1[o] = addm(mulm(x0[o], y1[o], q), mulm(x1[o], y0[o], q), q);
+            d2[o] = mulm(x1[o], y1[o], q);
+        }
+    }
+    return 0;
+}
+
+int or_relinearize(const or_params *P, const uint32_t *x0, const uint32_t *x1, const uint32_t *y0,
+                   const uint32_t *y1, uint32_t l, const uint8_t seed[32], const uint32_t *b,
+                   const uint32_t *a, int rounds, uint32_t *c0o, uint32_t *c1o) {
+    if (check_params(P, l)) return -1;
+    uint32_t N = 1u << P->logN;
+    size_t lN = (size_t)l * N;
+    uint32_t *d = (uint32_t *)malloc(sizeof(uint32_t) * 3 * lN);
+    uint32_t *k0 = (uint32_t *)malloc(sizeof(uint32_t) * lN);
+    int rc = or_tensor(P, x0, x1, y0, y1, l, d, d + lN, d + 2 * lN);
+    /* key switch of (0, d2): c0' = d0 + ob, c1' = d1 + oa */
+    if (!rc) {
+        memset(k0, 0, sizeof(uint32_t) * lN);
+        rc = or_keyswitch(P, k0, d + 2 * lN, l, seed, b, a, rounds, c0o, c1o);
+    }
+    if (!rc) {
+        for (uint32_t i = 0; i < l; i++) {
+            uint32_t q = P->q[i];
+            for (uint32_t n = 0; n < N; n++) {
+                size_t o = (size_t)i * N + n;
+                c0o[o] = addm(c0o[o], d[o], q);
+                c1o[o] = addm(c1o[o], d[lN + o], q);
+            }
+        }
+    }
+    free(k0);
+    free(d);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
 /* key generation (the oracle side only; the library never generates)  */
 /* ------------------------------------------------------------------ */
 

@@ -57,6 +57,15 @@ def lib():
         L.or_moddown.restype = i32
         L.or_keyswitch.argtypes = [vp, vp, vp, u32, vp, vp, vp, i32, vp, vp]
         L.or_keyswitch.restype = i32
+        L.or_automorph_ntt.argtypes = [vp, u32, u32, vp]
+        L.or_rotate.argtypes = [vp, vp, vp, u32, u32, vp, vp, vp, i32, vp, vp]
+        L.or_rotate.restype = i32
+        L.or_rotate_hoisted_one.argtypes = [vp, vp, vp, u32, u32, vp, vp, vp, i32, vp, vp]
+        L.or_rotate_hoisted_one.restype = i32
+        L.or_tensor.argtypes = [vp, vp, vp, vp, vp, u32, vp, vp, vp]
+        L.or_tensor.restype = i32
+        L.or_relinearize.argtypes = [vp, vp, vp, vp, vp, u32, vp, vp, vp, i32, vp, vp]
+        L.or_relinearize.restype = i32
         L.or_negacyclic_mul.argtypes = [vp, vp, u32, vp]
         L.or_automorph.argtypes = [vp, u32, u32, vp]
         L.or_ksk_gen.argtypes = [vp, vp, vp, vp, vp, i32, vp]
@@ -226,6 +235,82 @@ def keyswitch(P: Params, c0: np.ndarray, c1: np.ndarray, l: int, seed: bytes, b:
         ap = _p(a)
     if lib().or_keyswitch(P.ptr, _p(c0), _p(c1), l, _p(s), _p(b), ap, rounds, _p(c0o), _p(c1o)) != 0:
         raise ValueError("or_keyswitch: bad arguments")
+    return c0o, c1o
+
+
+def automorph_ntt(x: np.ndarray, logN: int, g: int) -> np.ndarray:
+    """X -> X^g on one NTT-domain limb (a slot permutation)."""
+    x = np.ascontiguousarray(x, dtype=np.uint32)
+    assert x.shape == (1 << logN,)
+    out = np.zeros_like(x)
+    lib().or_automorph_ntt(_p(x), logN, g, _p(out))
+    return out
+
+
+def rotate(P: Params, c0: np.ndarray, c1: np.ndarray, l: int, g: int, seed: bytes, b: np.ndarray,
+           a=None, rounds: int = ROUNDS):
+    """Key switch of (c0(X^g), c1(X^g)) with a key for s(X^g) -> s."""
+    c0 = np.ascontiguousarray(c0, dtype=np.uint32)
+    c1 = np.ascontiguousarray(c1, dtype=np.uint32)
+    b = np.ascontiguousarray(b, dtype=np.uint32)
+    assert c0.shape == (l, P.N) and c1.shape == (l, P.N)
+    c0o = np.zeros_like(c0)
+    c1o = np.zeros_like(c1)
+    ap = None
+    if a is not None:
+        a = np.ascontiguousarray(a, dtype=np.uint32)
+        ap = _p(a)
+    s = _seed(seed)
+    if lib().or_rotate(P.ptr, _p(c0), _p(c1), l, g, _p(s), _p(b), ap, rounds, _p(c0o), _p(c1o)) != 0:
+        raise ValueError("or_rotate: bad arguments")
+    return c0o, c1o
+
+
+def rotate_hoisted(P: Params, c0: np.ndarray, c1: np.ndarray, l: int, gs, seeds, bs,
+                   rounds: int = ROUNDS):
+    """Rotations of one ciphertext by each Galois element in gs, sharing one
+    ModUp of c1; returns [(c0', c1')] in the order of gs."""
+    c0 = np.ascontiguousarray(c0, dtype=np.uint32)
+    ext = modup(P, c1, l)
+    outs = []
+    for g, seed, b in zip(gs, seeds, bs):
+        b = np.ascontiguousarray(b, dtype=np.uint32)
+        c0o = np.zeros((l, P.N), dtype=np.uint32)
+        c1o = np.zeros((l, P.N), dtype=np.uint32)
+        s = _seed(seed)
+        if lib().or_rotate_hoisted_one(P.ptr, _p(c0), _p(ext), l, g, _p(s), _p(b), None, rounds,
+                                       _p(c0o), _p(c1o)) != 0:
+            raise ValueError("or_rotate_hoisted_one: bad arguments")
+        outs.append((c0o, c1o))
+    return outs
+
+
+def tensor(P: Params, x0, x1, y0, y1, l: int):
+    """(d0, d1, d2) of the product of ciphertexts (x0, x1) and (y0, y1)."""
+    xs = [np.ascontiguousarray(v, dtype=np.uint32) for v in (x0, x1, y0, y1)]
+    for v in xs:
+        assert v.shape == (l, P.N)
+    d = [np.zeros((l, P.N), dtype=np.uint32) for _ in range(3)]
+    if lib().or_tensor(P.ptr, *[_p(v) for v in xs], l, *[_p(v) for v in d]) != 0:
+        raise ValueError("or_tensor: bad arguments")
+    return tuple(d)
+
+
+def relinearize(P: Params, x0, x1, y0, y1, l: int, seed: bytes, b: np.ndarray, a=None,
+                rounds: int = ROUNDS):
+    """Tensor of two ciphertexts, then key switch of d2 with a key for s^2 -> s."""
+    xs = [np.ascontiguousarray(v, dtype=np.uint32) for v in (x0, x1, y0, y1)]
+    b = np.ascontiguousarray(b, dtype=np.uint32)
+    c0o = np.zeros((l, P.N), dtype=np.uint32)
+    c1o = np.zeros((l, P.N), dtype=np.uint32)
+    ap = None
+    if a is not None:
+        a = np.ascontiguousarray(a, dtype=np.uint32)
+        ap = _p(a)
+    s = _seed(seed)
+    if lib().or_relinearize(P.ptr, *[_p(v) for v in xs], l, _p(s), _p(b), ap, rounds,
+                            _p(c0o), _p(c1o)) != 0:
+        raise ValueError("or_relinearize: bad arguments")
     return c0o, c1o
 
 
