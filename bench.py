@@ -78,6 +78,27 @@ def workload_counts(logN: int, L: int, alpha: int, l: int, regen: bool = True):
     return {"modmuls": modmuls, "bytes": bytes_, "chacha_blocks": blocks}
 
 
+def op_counts(wl, l: int, regen: bool = True):
+    """Work of one step's unit of the workload's operation at level l: a key
+    switch or rotation (the automorphism is a permutation: no arithmetic), a
+    relinearisation (key switch + 4 slot products per coefficient, reading two
+    ciphertexts), or n_rot hoisted rotations (one ModUp, n_rot inner products
+    and ModDowns)."""
+    ks = workload_counts(wl.logN, wl.L, wl.alpha, l, regen)
+    N = 1 << wl.logN
+    if wl.op == "relin":
+        return {"modmuls": ks["modmuls"] + 4 * l * N, "bytes": ks["bytes"] + 2 * l * N * 4,
+                "chacha_blocks": ks["chacha_blocks"]}
+    if wl.op == "hoisted":
+        st = stage_modmuls(wl.logN, wl.L, wl.alpha, l)
+        up = st["intt_row_c1"] + st["modup_col"]
+        n = wl.n_rot
+        key_bytes = ks["bytes"] - 4 * l * N * 4
+        return {"modmuls": up + n * (ks["modmuls"] - up), "bytes": 2 * l * N * 4 + n * (key_bytes + 2 * l * N * 4),
+                "chacha_blocks": n * ks["chacha_blocks"]}
+    return ks
+
+
 def stage_modmuls(logN: int, L: int, alpha: int, l: int):
     """Modular multiplies done by each profiled stage (kernel) of one key switch."""
     N = 1 << logN
@@ -225,25 +246,43 @@ def run_ours(args):
         unit, metric = "key-switches/s", "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline"
         if args.workload == "sweep_n17":
             metric = "key-switches/s at N=2^17 level sweep 40..1 (1 B200)"
+        if wl.op in ("rotate", "hoisted"):
+            unit = "rotations/s"
+            metric = (f"rotations/s at N=2^{wl.logN} ({'single' if wl.op == 'rotate' else f'{wl.n_rot} hoisted'}"
+                      " rotation(s) per ciphertext; 1 B200)")
+        elif wl.op == "relin":
+            unit = "relinearisations/s"
+            metric = f"ciphertext products (tensor + relinearisation) per second at N=2^{wl.logN} (1 B200)"
         levels = list(wl.levels) if wl.levels else [L]
         B = wl.n_ct
+        nk = wl.n_rot if wl.op == "hoisted" else B  # keys per step
         ctx.ensure_workspace(max(levels), B)
-        per_set = (B * (2 * L * N * 4) + B * wl.dnum * (L + A) * N * 4 * (1 if regen else 2))
+        per_set = (B * (2 * L * N * 4) * (2 if wl.op == "relin" else 1)
+                   + nk * wl.dnum * (L + A) * N * 4 * (1 if regen else 2))
         nsets = max(2, math.ceil(2 * L2_BYTES / per_set)) if args.workload != "sweep_n17" else 1
         sets = []
+        nct = B * (2 if wl.op == "relin" else 1)
         for s in range(nsets):
-            keys = [make_key(1000 * s + k + 1) for k in range(B)]
+            keys = [make_key(1000 * s + k + 1) for k in range(nk)]
             ct = dev(np.stack([np.stack([synth.uniform_residues(q, N, 50 + s, rank, k, h) for h in range(2)])
-                               for k in range(B)]))
+                               for k in range(nct)]))
             sets.append((ct, keys))
-        out = torch.empty((B, 2, L, N), dtype=torch.int32, device="cuda")
-        units_per_step = B * len(levels)
+        out = torch.empty((max(B, wl.n_rot), 2, L, N), dtype=torch.int32, device="cuda")
+        units_per_step = (wl.n_rot if wl.op == "hoisted" else B) * len(levels)
+        rot_gs = [pow(5, 1 << r, 2 * N) for r in range(wl.n_rot)]  # steps 1, 2, 4, ...
 
         def step(k):
             ct, keys = sets[k % nsets]
             for l in levels:
                 lN = l * N
-                if B == 1:
+                if wl.op == "rotate":
+                    ctx.rotate(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs[0], keys[0], out[0, 0, :l], out[0, 1, :l],
+                               stream)
+                elif wl.op == "hoisted":
+                    ctx.rotate_hoisted(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs, keys, out[:, :, :l], stream)
+                elif wl.op == "relin":
+                    ctx.relinearize(ct[0, :, :l], ct[1, :, :l], l, keys[0], out[0, :, :l], stream)
+                elif B == 1:
                     # level-l ciphertext = the first l limbs of each half
                     c0 = ct[0, 0, :l]
                     c1 = ct[0, 1, :l]
@@ -253,7 +292,9 @@ def run_ours(args):
         # 6 launches per key switch (the inner product splits in two when the
         # ModDown branch overlaps), 5 in the instrumented (serial) calls
         launches_per_step = (5 if os.environ.get("PC_NO_OVERLAP") else 6) * len(levels)
-        work = [workload_counts(wl.logN, L, A, l, regen) for l in levels]
+        if wl.op == "hoisted":  # one ModUp (2), then per rotation 4 (3 when serial)
+            launches_per_step = (2 + (3 if os.environ.get("PC_NO_OVERLAP") else 4) * wl.n_rot) * len(levels)
+        work = [op_counts(wl, l, regen) for l in levels]
 
     # warm-up, then exactly K timed steps between barriers
     for k in range(args.warmup):
@@ -343,6 +384,16 @@ def run_ours(args):
                                               "modular multiply + 592 per ChaCha12 block"}
             res["stage_ms_per_step"] = {k: v / ncalls * len(levels) for k, v in stage_ms.items()}
             res["stage_sampling"] = f"{ncalls} of {args.steps * len(levels)} calls instrumented (every {PROF_EVERY}th)"
+        else:
+            # no per-kernel events on this path (hoisted rotations): the whole step
+            peak_ops = SMS * ISSUE_LANES_PER_SM_CLK * 1965e6
+            ops = (MODMUL_IMAD * mm + CHACHA_OPS * sum(w["chacha_blocks"] for w in work)) * wl.n_ct
+            ach = ops / sec_per_step
+            res["roofline"] = {"bound": "alu", "kernel": "whole step", "achieved": ach / 1e12,
+                               "peak": peak_ops / 1e12, "unit": "Tintop/s", "frac": ach / peak_ops,
+                               "traffic": None,
+                               "peak_source": "derived: 148 SMs x 128 issued 32-bit lane ops/clk x 1965 MHz; "
+                                              "ops = 4 per Shoup modular multiply + 592 per ChaCha12 block"}
 
     # end-to-end: host buffers through the same C-ABI call, copies timed
     if not args.no_e2e and args.workload in ("rot1_n16", "relin_n12"):
@@ -398,20 +449,45 @@ def _oracle_inputs(wl, q, p):
     return O, P, b, c0, c1, l, synth.chacha_seed(1, 0)
 
 
+def oracle_step(wl, O, P, b, c0, c1, l, seed):
+    """One unit batch of the workload's operation on the oracle; returns the
+    number of operations done (n_rot for hoisted rotations, else 1)."""
+    from key_switching_b200 import synth
+    if wl.op == "rotate":
+        O.rotate(P, c0, c1, l, pow(5, 1, 2 * P.N), seed, b)
+    elif wl.op == "hoisted":
+        gs = [pow(5, 1 << r, 2 * P.N) for r in range(wl.n_rot)]
+        O.rotate_hoisted(P, c0, c1, l, gs, [seed] * wl.n_rot, [b] * wl.n_rot)
+        return wl.n_rot
+    elif wl.op == "relin":
+        y0 = synth.uniform_residues(P.q[:l], P.N, 51, 0, 0, 0)
+        y1 = synth.uniform_residues(P.q[:l], P.N, 51, 0, 0, 1)
+        O.relinearize(P, c0, c1, y0, y1, l, seed, b)
+    else:
+        O.keyswitch(P, c0, c1, l, seed, b)
+    return 1
+
+
+def _unit(wl):
+    return {"rotate": "rotations/s", "hoisted": "rotations/s", "relin": "relinearisations/s"}.get(
+        wl.op, "key-switches/s")
+
+
 def cpu_baseline(wl, q, p, budget_s: float = 20.0):
     """The oracle as it stands, single-threaded, on a bounded sample: as many
-    full key switches of the workload as fit in about budget_s seconds."""
+    full operations of the workload as fit in about budget_s seconds."""
     O, P, b, c0, c1, l, seed = _oracle_inputs(wl, q, p)
     t0 = time.perf_counter()
-    n = 0
+    n = ops = 0
     while True:
-        O.keyswitch(P, c0, c1, l, seed, b)
+        ops += oracle_step(wl, O, P, b, c0, c1, l, seed)
         n += 1
         if time.perf_counter() - t0 >= budget_s or n >= 50:
             break
     dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "key-switches/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} full key switch(es) of {wl.name} (l={l}) in {dt:.1f} s, single thread"}
+    return {"value": ops / dt, "unit": _unit(wl), "cores": 1, "kind": "oracle",
+            "sample": f"{n} full {wl.op} step(s) ({ops} operation(s)) of {wl.name} (l={l}) in {dt:.1f} s, "
+                      "single thread"}
 
 
 def run_reference(args):
@@ -425,24 +501,33 @@ def run_reference(args):
     budget = args.cpu_budget * 6
     t0 = time.perf_counter()
     for _ in range(min(args.warmup, 1)):
-        O.keyswitch(P, c0, c1, l, seed, b)
+        oracle_step(wl, O, P, b, c0, c1, l, seed)
     t_one = max(1e-3, time.perf_counter() - t0)
     steps = max(1, min(args.steps, int(budget / t_one)))
     t0 = time.perf_counter()
+    ops = 0
     for _ in range(steps):
-        O.keyswitch(P, c0, c1, l, seed, b)
+        ops += oracle_step(wl, O, P, b, c0, c1, l, seed)
     dt = time.perf_counter() - t0
-    v = steps / dt
-    unit = "key-switches/s"
-    res = {"impl": "reference", "metric": "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline",
+    v = ops / dt
+    unit = _unit(wl)
+    metric = "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline"
+    if wl.op in ("rotate", "hoisted"):
+        metric = (f"rotations/s at N=2^{wl.logN} ({'single' if wl.op == 'rotate' else f'{wl.n_rot} hoisted'}"
+                  " rotation(s) per ciphertext; 1 B200)")
+    elif wl.op == "relin":
+        metric = f"ciphertext products (tensor + relinearisation) per second at N=2^{wl.logN} (1 B200)"
+    elif wl.name == "sweep_n17":
+        metric = "key-switches/s at N=2^17 level sweep 40..1 (1 B200)"
+    res = {"impl": "reference", "metric": metric,
            "value": v, "unit": unit, "n_gpus": 1, "steps": steps, "warmup": min(args.warmup, 1),
            "ms_per_step": dt * 1e3 / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "u32", "data": "synthetic",
            "config": {"workload": f"{wl.name}: N=2^{wl.logN}, L={wl.L}, alpha={wl.alpha}, dnum={wl.dnum}, "
                       "1 ct/step at the top level, key a-half regenerated (ChaCha12)"},
            "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle",
-                            "sample": f"{steps} of {args.steps} requested step(s), each one full key switch, "
-                                      "time-bounded, single thread"},
+                            "sample": f"{steps} of {args.steps} requested step(s), each one full {wl.op} "
+                                      f"({ops} operation(s) in all), time-bounded, single thread"},
            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
@@ -454,7 +539,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="rot1_n16",
-                    choices=["rot1_n16", "relin_n12", "batch16_n16", "ntt_n16", "sweep_n17"])
+                    choices=["rot1_n16", "relin_n12", "batch16_n16", "ntt_n16", "sweep_n17", "rotate_n16",
+                             "hoisted8_n16", "relin_mul_n12", "relin_mul_n16"])
     ap.add_argument("--keys", default="regen", choices=["regen", "stored"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

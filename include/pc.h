@@ -171,6 +171,45 @@ int pc_keyswitch(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l
 int pc_keyswitch_batch(pc_ctx *ctx, const uint32_t *ct, uint32_t B, uint32_t l,
                        const pc_ksk *keys, uint32_t *out, pc_stream stream);
 
+/* Rotation: the key switch of c(X^g) = (c0(X^g), c1(X^g)) -- the ciphertext
+ * under the automorphism X -> X^g, which decrypts under s(X^g) -- with a key
+ * k for s(X^g) -> s.  (Perseus README, "Python API": the session holds keys
+ * for the rotations a model uses, e.g. steps 1, 2, 4, 8, and
+ * fhe.rotate_and_sum rotates by them; the pages give no formula, so this is
+ * the textbook CKKS rotation: automorphism, then key switch.)  galois = g,
+ * odd and < 2N (5^r mod 2N rotates the slots by r; 2N-1 conjugates), else
+ * PC_E_ARG.  In the NTT domain X -> X^g permutes the slots: slot k of
+ * x(X^g) is slot k' of x with 2 brv(k') + 1 = g (2 brv(k) + 1) mod 2N; the
+ * kernels apply it while reading c1 and c0 (no permuted copy is made).
+ * c0, c1, c0o, c1o: device [l][N] NTT; the outputs must not overlap the
+ * inputs (PC_E_ARG).  Needs the workspace for (l, 1). */
+int pc_rotate(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t galois,
+              const pc_ksk *k, uint32_t *c0o, uint32_t *c1o, pc_stream stream);
+
+/* Hoisted rotations of one ciphertext by n Galois elements (the rotations of
+ * one fhe.rotate_and_sum-style step list): ModUp of c1 runs once; rotation i
+ * applies X -> X^galois[i] to the extended limbs ext_j inside the inner product
+ * (a permuted ModUp output is a valid lift of c1(X^g)), then ModDown and
+ * c0(X^g) as in pc_rotate.  galois, keys: host arrays of n (1 <= n <= 64);
+ * keys[i] switches s(X^galois[i]) -> s.  out: device [n][2][l][N], rotation i
+ * at out + 2 i l N (c0' then c1'), not overlapping c0 or c1.  Results equal
+ * the hoisted oracle bit for bit; they differ from pc_rotate's only in the
+ * ModUp approximation term, and both decrypt within the same bound.  Needs
+ * the workspace for (l, 1). */
+int pc_rotate_hoisted(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t n,
+                      const uint32_t *galois, const pc_ksk *keys, uint32_t *out, pc_stream stream);
+
+/* Relinearisation of a ciphertext product (Perseus README, "Python API":
+ * fhe.square; the textbook CKKS multiplication): the tensor of x = (x0, x1)
+ * and y = (y0, y1) is (d0, d1, d2) = (x0 y0, x0 y1 + x1 y0, x1 y1) slot-wise
+ * mod q_i (d0 + d1 s + d2 s^2 decrypts to the product), and d2 is key-switched
+ * with a key k for s^2 -> s: out = (d0 + ModDown_b, d1 + ModDown_a).  The
+ * tensor terms are formed inside the kernels that read x and y.  x, y, out:
+ * device [2][l][N] NTT; out must not overlap x or y (PC_E_ARG); x may equal
+ * y (squaring).  Needs the workspace for (l, 1). */
+int pc_relinearize(pc_ctx *ctx, const uint32_t *x, const uint32_t *y, uint32_t l, const pc_ksk *k,
+                   uint32_t *out, pc_stream stream);
+
 /* Test hook: write the regenerated 'a' words for level l.  a_out: device
  * [beta][l+alpha][N], a_out[j][t][k] = a_{j,g(t)}[k] where (spec v1) block
  * b = k/8 of ChaCha12 with state words (constants "expand 32-byte k", seed as

@@ -117,8 +117,8 @@ struct DeviceGuard {
 
 // workspace regions for B ciphertexts at level l (words)
 struct Layout {
-    size_t w1, t, acc, u, total;  // offsets and total, in words
-    size_t w1z, tz, accz, uz;     // per-ciphertext strides
+    size_t w1, t, acc, u, x, total;  // offsets and total, in words
+    size_t w1z, tz, accz, uz, xz;    // per-ciphertext strides
 };
 Layout layout(const pc_ctx *c, u32 l, u32 B) {
     Layout L{};
@@ -131,7 +131,11 @@ Layout layout(const pc_ctx *c, u32 l, u32 B) {
     L.t = L.w1 + B * L.w1z;
     L.acc = L.t + B * L.tz;
     L.u = L.acc + B * L.accz;
-    L.total = L.u + B * L.uz;
+    // X: c1 as the ModUp read it (rotated, or relinearisation's d2), for the
+    // own-digit limbs of the inner product
+    L.xz = l * N;
+    L.x = L.u + B * L.uz;
+    L.total = L.x + B * L.xz;
     return L;
 }
 
@@ -509,26 +513,64 @@ int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_str
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
-// shared body of pc_keyswitch and pc_keyswitch_batch: B ciphertexts whose
-// c0 / c1 / outputs sit at stride `cz` words.
-static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u32 l, const pc_ksk *keys,
-                          u32 B, u32 *o0, u32 *o1, cudaStream_t s) {
+// How the kernels read a key switch's inputs.  galois != 1: the automorphism
+// X -> X^galois is applied to c1 (ModUp input and own-digit limbs) and c0 as
+// they are read; rot: it is applied to the extended limbs instead (hoisted
+// rotation; ModUp of the unrotated c1 already in the workspace); mul: c1 is
+// the slot-wise product c1 * mul (relinearisation's d2); rx, ry: the tensor
+// terms d0, d1 of ciphertexts rx, ry are added to the outputs instead of c0.
+struct KsInput {
+    u32 galois = 1, ginv = 1;
+    bool rot = false;
+    const u32 *mul = nullptr, *rx = nullptr, *ry = nullptr;
+};
+
+// x^-1 mod 2N for odd x (Newton iteration on the 2-adic inverse).
+static u32 inv_mod_2n(u32 x, u32 N) {
+    u32 y = x;  // x * x = 1 mod 8
+    for (int i = 0; i < 5; ++i) y *= 2u - x * y;
+    return y & (2u * N - 1u);
+}
+
+static bool galois_ok(const pc_ctx *c, u32 g) { return (g & 1u) && g < 2u * c->N; }
+
+// events of an instrumented call, or null (measurement only)
+static cudaEvent_t *profile_slot(pc_ctx *c) {
+    if (c->prof_ev && c->prof_used < c->prof_max && (c->prof_seen++ % c->prof_every) == 0)
+        return c->prof_ev + (size_t)(c->prof_used++) * (PC_PROFILE_STAGES + 1);
+    return nullptr;
+}
+
+// ModUp up to the column-pass output T in the workspace: inverse row pass of
+// c1 (through the input transform), then the conversion kernel.
+static cudaError_t ks_modup(pc_ctx *c, const u32 *c1, size_t cz, u32 l, u32 B, const KsInput &in, cudaStream_t s,
+                            cudaEvent_t *ev) {
     const Layout Lw = layout(c, l, B);
     u32 *ws = (u32 *)c->ws;
-    u32 *w1 = ws + Lw.w1, *wt = ws + Lw.t, *wacc = ws + Lw.acc, *wu = ws + Lw.u;
-    const bool regen = keys[0].a == nullptr;
-    for (u32 b = 1; b < B; ++b)
-        if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
-    // optional per-stage events (measurement only)
-    cudaEvent_t *ev = nullptr;
-    if (c->prof_ev && c->prof_used < c->prof_max && (c->prof_seen++ % c->prof_every) == 0)
-        ev = c->prof_ev + (size_t)(c->prof_used++) * (PC_PROFILE_STAGES + 1);
     auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
     mark(0);
-    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, B, cz, Lw.w1z, false, true, s);
+    const bool xform = (in.galois != 1 && !in.rot) || in.mul;  // c1 is read transformed
+    cudaError_t e = pc::launch_row(c, false, c1, ws + Lw.w1, 0, l, B, cz, Lw.w1z, false, true, s,
+                                   in.rot ? 1u : in.galois, in.mul, xform ? ws + Lw.x : nullptr);
     mark(1);
-    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, Lw.w1z, wt, Lw.tz, l, B, true, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, ws + Lw.w1, Lw.w1z, ws + Lw.t, Lw.tz, l, B, true, s);
     mark(2);
+    return e;
+}
+
+// Inner products, ModDown and the output combination, from T in the workspace.
+static cudaError_t ks_finish(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u32 l, const pc_ksk *keys, u32 B,
+                             u32 *o0, u32 *o1, const KsInput &in, cudaStream_t s, cudaEvent_t *ev) {
+    const Layout Lw = layout(c, l, B);
+    u32 *ws = (u32 *)c->ws;
+    u32 *wt = ws + Lw.t, *wacc = ws + Lw.acc, *wu = ws + Lw.u;
+    const bool regen = keys[0].a == nullptr;
+    auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
+    cudaError_t e = cudaSuccess;
+    // own-digit limbs: c1 itself, or the transformed copy ks_modup stored
+    const bool xform = (in.galois != 1 && !in.rot) || in.mul;
+    const u32 *own = xform ? ws + Lw.x : c1;
+    const size_t ownz = xform ? Lw.xz : cz;
     // The ModDown branch needs only the special-prime accumulators: when not
     // instrumented, those inner products run first on the high-priority
     // internal stream, followed there by the ModDown conversion kernel, while
@@ -544,12 +586,12 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
                 kp.a[i] = keys[b0 + i].a;
                 seed_words(keys[b0 + i].seed, kp.seed[i]);
             }
-            e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, c1 + b0 * cz, cz, wacc + b0 * Lw.accz, Lw.accz, l,
-                                 kp, nb, regen, true, st, t0, nt);
+            e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, own + b0 * ownz, ownz, wacc + b0 * Lw.accz,
+                                 Lw.accz, l, kp, nb, regen, true, st, t0, nt, in.galois, in.ginv, in.rot);
         }
     };
     if (fork) {
-        if (e == cudaSuccess) e = cudaEventRecord(c->ev_fork, s);
+        e = cudaEventRecord(c->ev_fork, s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(c->aux, c->ev_fork, 0);
         inner(c->aux, l, c->alpha);
         if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, true, c->aux);
@@ -562,9 +604,30 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
         if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, true, s);
     }
     mark(4);
-    if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, c0, cz, o0, o1, cz, l, B, s);
+    if (e == cudaSuccess)
+        e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, in.rx ? nullptr : c0, cz, o0, o1, cz, l, B, s,
+                                   in.galois, in.rx, in.ry);
     mark(5);
+    return e;
+}
+
+// shared body of the key-switching calls: B ciphertexts whose c0 / c1 /
+// outputs sit at stride `cz` words.
+static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u32 l, const pc_ksk *keys,
+                          u32 B, u32 *o0, u32 *o1, cudaStream_t s, const KsInput &in = KsInput{}) {
+    const bool regen = keys[0].a == nullptr;
+    for (u32 b = 1; b < B; ++b)
+        if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
+    cudaEvent_t *ev = profile_slot(c);
+    cudaError_t e = ks_modup(c, c1, cz, l, B, in, s, ev);
+    if (e == cudaSuccess) e = ks_finish(c, c0, c1, cz, l, keys, B, o0, o1, in, s, ev);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+// do [a, a + an) and [b, b + bn) intersect
+static bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return x < y + bn && y < x + an;
 }
 
 int pc_keyswitch(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
@@ -587,6 +650,67 @@ int pc_keyswitch_batch(pc_ctx *c, const uint32_t *ct, uint32_t B, uint32_t l, co
     DeviceGuard dg(c->device);
     const size_t lN = (size_t)l * c->N;
     return keyswitch_core(c, ct, ct + lN, 2 * lN, l, keys, B, out, out + lN, (cudaStream_t)stream);
+}
+
+int pc_rotate(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t galois, const pc_ksk *k,
+              uint32_t *c0o, uint32_t *c1o, pc_stream stream) {
+    if (!c || !c0 || !c1 || !c0o || !c1o || l < 1 || l > c->L || !galois_ok(c, galois)) return PC_E_ARG;
+    if (int r = check_ksk(c, k)) return r;
+    if (!aligned16(c0) || !aligned16(c1) || !aligned16(c0o) || !aligned16(c1o)) return PC_E_ALIGN;
+    const size_t lb = (size_t)l * c->N * sizeof(u32);
+    // the automorphism reads other rows than it writes: no in-place outputs
+    if (overlaps(c0o, lb, c0, lb) || overlaps(c0o, lb, c1, lb) || overlaps(c1o, lb, c0, lb) ||
+        overlaps(c1o, lb, c1, lb))
+        return PC_E_ARG;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    KsInput in;
+    in.galois = galois;
+    return keyswitch_core(c, c0, c1, 0, l, k, 1, c0o, c1o, (cudaStream_t)stream, in);
+}
+
+int pc_rotate_hoisted(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t n,
+                      const uint32_t *galois, const pc_ksk *keys, uint32_t *out, pc_stream stream) {
+    if (!c || !c0 || !c1 || !out || !galois || !keys || l < 1 || l > c->L || n < 1 || n > 64) return PC_E_ARG;
+    for (u32 i = 0; i < n; ++i) {
+        if (!galois_ok(c, galois[i])) return PC_E_ARG;
+        if (int r = check_ksk(c, &keys[i])) return r;
+    }
+    if (!aligned16(c0) || !aligned16(c1) || !aligned16(out)) return PC_E_ALIGN;
+    const size_t lN = (size_t)l * c->N, ob = 2 * (size_t)n * lN * sizeof(u32);
+    if (overlaps(out, ob, c0, lN * sizeof(u32)) || overlaps(out, ob, c1, lN * sizeof(u32))) return PC_E_ARG;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = ks_modup(c, c1, 0, l, 1, KsInput{}, s, nullptr);
+    for (u32 i = 0; e == cudaSuccess && i < n; ++i) {
+        KsInput in;
+        in.galois = galois[i];
+        in.ginv = inv_mod_2n(galois[i], c->N);
+        if (((in.galois * in.ginv) & (2u * c->N - 1u)) != 1u) return PC_E_ARG;  // cannot happen for odd g
+        in.rot = true;
+        u32 *o = out + 2 * (size_t)i * lN;
+        e = ks_finish(c, c0, c1, 0, l, &keys[i], 1, o, o + lN, in, s, nullptr);
+    }
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+int pc_relinearize(pc_ctx *c, const uint32_t *x, const uint32_t *y, uint32_t l, const pc_ksk *k, uint32_t *out,
+                   pc_stream stream) {
+    if (!c || !x || !y || !out || l < 1 || l > c->L) return PC_E_ARG;
+    if (int r = check_ksk(c, k)) return r;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(out)) return PC_E_ALIGN;
+    const size_t lN = (size_t)l * c->N;
+    const size_t cb = 2 * lN * sizeof(u32);
+    if (overlaps(out, cb, x, cb) || overlaps(out, cb, y, cb)) return PC_E_ARG;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    // key switch of d2 = x1 y1; d0 and d1 are formed in the final kernel
+    KsInput in;
+    in.mul = y + lN;
+    in.rx = x;
+    in.ry = y;
+    return keyswitch_core(c, nullptr, x + lN, 0, l, k, 1, out, out + lN, (cudaStream_t)stream, in);
 }
 
 int pc_expand_a(pc_ctx *c, const uint8_t seed[32], uint32_t l, uint32_t *a_out, pc_stream stream) {

@@ -88,6 +88,48 @@ struct LastPhase {
 struct RowAddr {
     __device__ __forceinline__ int operator()(int x) const { return x + (x >> 4); }
 };
+
+// ------------------------------------------- automorphisms and slot products
+// X -> X^g (g odd) on an NTT-domain limb is a slot permutation: slot k holds
+// the value at psi^(2 brv(k) + 1), so slot k of x(X^g) is slot k' of x with
+// 2 brv(k') + 1 = g (2 brv(k) + 1) mod 2N.  In the R x C view every row goes
+// to a single row and every aligned block of 8 rows to an aligned block.
+template <int LOGN>
+__device__ __forceinline__ u32 auto_src(u32 k, u32 g) {
+    const u32 idx = __brev(k) >> (32 - LOGN);
+    const u32 e = (g * (2u * idx + 1u)) & ((2u << LOGN) - 1u);  // mod 2N (a power of two)
+    return __brev(e >> 1) >> (32 - LOGN);
+}
+
+// a b mod q, canonical, for a, b < q: REDC of the product gives a b 2^-32.
+__device__ __forceinline__ u32 mulmod(u32 a, u32 b, const PrimeK &pk) {
+    const u64 p = (u64)a * b;
+    return shoup(redc((u32)p, (u32)(p >> 32), pk.q, pk.qn), pk.r32, pk.r32s, pk.q);
+}
+
+// Elements x_of(lt, r) (layout PH) of row `row` of the limb x(X^g) (g = 1:
+// x itself), times the same elements of y(X^g) when y is given (the slot-wise
+// product of a ciphertext tensor).  Inputs canonical.
+template <class PH, int LOGN, int C>
+__device__ __forceinline__ void load_row_in(u32 v[16], const u32 *x, const u32 *y, int row, int lt, u32 g,
+                                            const PrimeK &pk) {
+    if (g == 1) {
+        gload<PH>(v, x + (size_t)row * C, lt);
+        if (y) {
+            u32 w[16];
+            gload<PH>(w, y + (size_t)row * C, lt);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) v[r] = mulmod(v[r], w[r], pk);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const u32 k = auto_src<LOGN>((u32)(row * C + PH::x_of(lt, r)), g);
+            v[r] = __ldg(x + k);
+            if (y) v[r] = mulmod(v[r], __ldg(y + k), pk);
+        }
+    }
+}
 template <int W>
 struct ColAddr {
     int c;
@@ -152,7 +194,8 @@ constexpr size_t row_smem_bytes(int tiles) {
 // place allowed), or for CMOUT (inverse only) column-major limbs.
 template <int LOGN, bool FWD, bool CMOUT>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
-k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int canonical) {
+k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int canonical, u32 galois,
+      const u32 *mul, u32 *xout) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -165,18 +208,26 @@ k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
     const int rho = threadIdx.x / GE::TPR, lt = threadIdx.x % GE::TPR;
     const int row0 = blockIdx.x * GE::NL, row = row0 + rho;
     const u32 g = first_prime + blockIdx.y;
-    const u32 q = T.pk[g].q;
+    const PrimeK pk = T.pk[g];
+    const u32 q = pk.q;
     stage_row_tw<GE>(stw, (FWD ? T.rowF : T.rowI) + (size_t)g * GE::N + (size_t)row0 * GE::C);
     pdl_wait();
     pdl_trigger();
     const size_t limb = (size_t)blockIdx.y * GE::N;
-    const u32 *src = in + blockIdx.z * zin + limb + (size_t)row * GE::C;
+    const u32 *src = in + blockIdx.z * zin + limb;
     u32 *dst = out + blockIdx.z * zout + limb;
     u32 v[16];
     u32 *line = sm + rho * GE::ROW_LS;
     const TwRow tw{stw + rho * GE::C};
-    if constexpr (FWD) gload<PF>(v, src, lt);
-    else gload<PLAST>(v, src, lt);
+    // the inverse pass reads a ciphertext limb, optionally through an
+    // automorphism and / or times a second limb (relinearisation's d2)
+    if constexpr (FWD) {
+        gload<PF>(v, src + (size_t)row * GE::C, lt);
+    } else {
+        load_row_in<PLAST, LOGN, GE::C>(v, src, mul ? mul + blockIdx.z * zin + limb : nullptr, row, lt, galois, pk);
+        // the transformed input itself (row-major, stride zout) for later readers
+        if (xout) gstore<PLAST>(v, xout + blockIdx.z * zout + limb + (size_t)row * GE::C, lt);
+    }
     cp_async_wait_all();
     __syncthreads();
     if constexpr (FWD) line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
@@ -380,6 +431,207 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
 // REGEN: a from ChaCha12 (spec v1), else from the stored key.
 // PINTT: special-prime limbs get the inverse row pass and are stored
 // column-major (the ModDown column kernel reads them so).
+// k_inner_rot (hoisted rotation, fused): ext_j is replaced by
+// ext_j(X^galois).  Each thread-row loads a source row of the block that the
+// automorphism maps onto this CTA's output rows (for a converted limb it runs
+// the row pass on it), then permutes the row's columns through shared memory
+// into its output row; ginv = galois^-1 mod 2N.  Its body, inner_body, also
+// covers ROT = false, but k_inner keeps a text of its own: instantiated from
+// the shared body, ptxas scheduled the plain kernel's loads later (twice the
+// long-scoreboard stalls at the same instruction count; 84 instead of 80 us
+// at N=2^16, l=24).
+enum { XF_PLAIN = 0, XF_GATHER = 1, XF_MUL = 3 };  // input modes of the ModDown finish
+template <int LOGN, bool FUSED, bool REGEN, bool ROT>
+__device__ __forceinline__ void inner_body(const Tables &T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
+                                           u32 *acc, size_t accz, u32 l, const KeyPack &kp, int pintt, u32 t0,
+                                           u32 galois, u32 ginv) {
+    static_assert(FUSED || !ROT, "rotation of the extended limbs needs the fused row pass");
+    using GE = Geo<LOGN>;
+    using PL = Plan<GE::LOGC>;
+    using PF = typename PL::P0;
+    using PLAST = typename LastPhase<GE::LOGC>::type;
+    extern __shared__ __align__(16) u32 dyn[];
+    uint2 *stw = reinterpret_cast<uint2 *>(dyn);           // [NL][C] row twiddles
+    u32 *sm = dyn + 2 * GE::NL * GE::C;                      // [NL][ROW_LS] exchange
+    u32 *tiles = sm + GE::NL * GE::ROW_LS;                   // [2][C*8] staging
+    const int rho = threadIdx.x / GE::TPR, lt = threadIdx.x % GE::TPR;
+    const int row0 = blockIdx.x * GE::NL;
+    const u32 t = t0 + blockIdx.y, z = blockIdx.z;
+    const u32 ll = l + T.alpha, beta = (l + T.alpha - 1) / T.alpha;
+    const u32 g = glob_of(T, l, t);
+    const PrimeK pk = T.pk[g];
+    const u32 q = pk.q;
+    // thread-row rho runs the row pass of source row srow0 + rho and
+    // accumulates output row orow (the same row unless ROT)
+    int srow0 = row0, orow = row0 + rho;
+    // ROT: source column of each of the thread's output elements, 8 bits each,
+    // after the staging tiles in dynamic shared memory
+    u32 *scol = tiles + 2 * GE::C * 8;
+    if constexpr (ROT) {
+        static_assert(GE::C <= 256, "source columns are packed in bytes");
+        srow0 = (int)(auto_src<LOGN>((u32)row0 * GE::C, galois) / GE::C) & ~(GE::NL - 1);
+        orow = (int)(auto_src<LOGN>((u32)(srow0 + rho) * GE::C, ginv) / GE::C);
+        u32 cs[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const u32 k = auto_src<LOGN>((u32)(orow * GE::C + PLAST::x_of(lt, r)), galois);
+            cs[r >> 2] |= (k & (GE::C - 1)) << (8 * (r & 3));
+        }
+        *reinterpret_cast<uint4 *>(scol + 4 * threadIdx.x) = make_uint4(cs[0], cs[1], cs[2], cs[3]);
+    }
+    const size_t rowoff = (size_t)orow * GE::C;
+    u32 *line = sm + rho * GE::ROW_LS;
+    const TwRow tw{stw + rho * GE::C};
+    const u32 jown = t < l ? t / T.alpha : beta;  // the digit holding t, if any
+    if (FUSED) stage_row_tw<GE>(stw, T.rowF + (size_t)g * GE::N + (size_t)srow0 * GE::C);
+    // counter-free quarter rounds of every digit's ChaCha12 blocks, once per CTA
+    __shared__ __align__(16) u32 spre[12 * MAX_L];
+    if (REGEN && threadIdx.x < beta) {
+        u32 sd[8], pre[12];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sd[i] = kp.seed[z][i];
+        chacha12_precolumn(sd, g, threadIdx.x, pre);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) spre[12 * threadIdx.x + i] = pre[i];
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+    const u32 *srcz_p = src + z * srcz;
+    u32 jn = (jown == 0) ? 1 : 0;  // next converted digit to stage
+    int buf = 0;
+    if (FUSED && jn < beta) stage_cm_rows<GE>(tiles, srcz_p + ((size_t)jn * ll + t) * GE::N, srow0);
+    u32 seed[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) seed[i] = kp.seed[z][i];
+    const u32 *kb = kp.b[z];
+    const u32 *ka = kp.a[z];
+    const size_t LLN = (size_t)(T.L + T.alpha) * GE::N;
+
+    u64 sb[16], sa[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) { sb[r] = 0; sa[r] = 0; }
+
+    for (u32 j = 0; j < beta; ++j) {
+        const bool own = j == jown;
+        u32 v[16], bv[16], av[16];
+        if (FUSED && !own) {
+            // this digit's tile has landed for every thread; the other tile's
+            // readers (previous converted digit) are done: prefetch the next
+            cp_async_wait_all();
+            __syncthreads();
+            jn = j + 1 + ((j + 1) == jown ? 1 : 0);
+            if (jn < beta)
+                stage_cm_rows<GE>(tiles + (buf ^ 1) * GE::C * 8, srcz_p + ((size_t)jn * ll + t) * GE::N, srow0);
+            const u32 *tl = tiles + buf * GE::C * 8;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) v[r] = tl[cm_addr(PF::x_of(lt, r), rho)];
+            buf ^= 1;
+        } else if (FUSED) {
+            // own digit: the input limb itself (ROT: its source row, permuted below)
+            gload<PLAST>(v, c1 + z * c1z + (size_t)t * GE::N + (size_t)(ROT ? srow0 + rho : orow) * GE::C, lt);
+        } else {
+            gload<PLAST>(v, srcz_p + ((size_t)j * ll + t) * GE::N + rowoff, lt);
+        }
+        gload<PLAST>(bv, kb + (size_t)j * LLN + (size_t)g * GE::N + rowoff, lt);
+        if constexpr (!REGEN) gload<PLAST>(av, ka + (size_t)j * LLN + (size_t)g * GE::N + rowoff, lt);
+        // regenerate a_{j,g} (pure ALU work, overlaps the loads above): the
+        // thread's elements form groups of KK consecutive coefficients
+        if constexpr (REGEN && PLAST::KK == 16) {
+            // the thread's 16 consecutive coefficients are two whole blocks
+            const u32 base = (u32)(rowoff + PLAST::x_of(lt, 0));
+            u32 o0[16], o1[16];
+            u32 pre[12];
+            const uint4 *pp = reinterpret_cast<const uint4 *>(spre + 12 * j);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const uint4 w4 = pp[i];
+                pre[4 * i] = w4.x; pre[4 * i + 1] = w4.y; pre[4 * i + 2] = w4.z; pre[4 * i + 3] = w4.w;
+            }
+            chacha12_block2_pre(pre, seed, base >> 3, g, j, o0, o1);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                av[w] = redc(o0[2 * w], mod32(o0[2 * w + 1], q, pk.q1s), q, pk.qn);
+                av[8 + w] = redc(o1[2 * w], mod32(o1[2 * w + 1], q, pk.q1s), q, pk.qn);
+            }
+        } else if constexpr (REGEN) {
+#pragma unroll
+            for (int gi = 0; gi < PLAST::G; ++gi) {
+                const u32 base = (u32)(rowoff + PLAST::x_of(lt, gi * PLAST::KK));
+#pragma unroll
+                for (int bb = 0; bb < (PLAST::KK + 7) / 8; ++bb) {
+                    u32 ks[16];
+                    const u32 k0 = base + bb * 8;
+                    chacha12_block(seed, k0 >> 3, g, j, ks);
+#pragma unroll
+                    for (int w = 0; w < 8 && bb * 8 + w < PLAST::KK; ++w) {
+                        const u32 wi = (k0 + w) & 7;
+                        // a * 2^-32 mod q from the 64-bit word pair
+                        av[gi * PLAST::KK + bb * 8 + w] = redc(ks[2 * wi], mod32(ks[2 * wi + 1], q, pk.q1s), q, pk.qn);
+                    }
+                }
+            }
+        }
+        if (FUSED && !own) line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
+        if constexpr (ROT) {
+            // column x of output row orow is column colsrc of the source row
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < 16; ++r) line[RowAddr{}(PLAST::x_of(lt, r))] = v[r];
+            __syncwarp();
+            const uint4 c4 = *reinterpret_cast<const uint4 *>(scol + 4 * threadIdx.x);
+            const u32 colsrc[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int r = 0; r < 16; ++r) v[r] = line[RowAddr{}((int)((colsrc[r >> 2] >> (8 * (r & 3))) & 0xffu))];
+            __syncwarp();
+        }
+        // multiply-accumulate; fold the 64-bit sums every two digits
+        const bool fold = (j & 1) && (j + 1 < beta);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const u32 e = red1(v[r], q);
+            sb[r] += (u64)e * bv[r];
+            sa[r] += (u64)e * av[r];
+            if (fold) {
+                sb[r] = fold64(sb[r], q, pk.q1s);
+                sa[r] = fold64(sa[r], q, pk.q1s);
+            }
+        }
+    }
+    // canonical sums: REDC divides by 2^32; regenerated a carries another 2^-32
+    u32 ob[16], oa[16];
+    const u32 ca = REGEN ? pk.r64 : pk.r32, cas = REGEN ? pk.r64s : pk.r32s;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        ob[r] = shoup(redc64(sb[r], q, pk.qn, pk.q1s), pk.r32, pk.r32s, q);
+        oa[r] = shoup(redc64(sa[r], q, pk.qn, pk.q1s), ca, cas, q);
+    }
+    u32 *d0 = acc + z * accz + (size_t)t * GE::N;
+    u32 *d1 = acc + z * accz + (size_t)(ll + t) * GE::N;
+    if (pintt && t >= l) {
+        cp_async_wait_all();
+        __syncthreads();  // every reader of the forward table and the tiles is done
+        stage_row_tw<GE>(stw, T.rowI + (size_t)g * GE::N + (size_t)row0 * GE::C);
+        cp_async_wait_all();
+        __syncthreads();
+        const TwRow twi{stw + (orow - row0) * GE::C};  // twiddles of the output row
+        line_inv<GE::LOGC>(ob, line, lt, RowAddr{}, twi, q, SyncWarp{});
+        line_inv<GE::LOGC>(oa, line, lt, RowAddr{}, twi, q, SyncWarp{});
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int a = cm_addr(PF::x_of(lt, r), orow - row0);
+            tiles[a] = ob[r];
+            tiles[GE::C * 8 + a] = oa[r];
+        }
+        __syncthreads();
+        store_cm_rows<GE>(tiles, d0, row0);
+        store_cm_rows<GE>(tiles + GE::C * 8, d1, row0);
+    } else {
+        gstore<PLAST>(ob, d0 + rowoff, lt);
+        gstore<PLAST>(oa, d1 + rowoff, lt);
+    }
+}
+
 template <int LOGN, bool FUSED, bool REGEN>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 4)
 k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz,
@@ -537,14 +789,25 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
     }
 }
 
+template <int LOGN, bool REGEN>
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 4)
+k_inner_rot(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
+            KeyPack kp, int pintt, u32 t0, u32 galois, u32 ginv) {
+    inner_body<LOGN, true, REGEN, true>(T, src, srcz, c1, c1z, acc, accz, l, kp, pintt, t0, galois, ginv);
+}
+
 // ----------------------------------------------------------- ModDown finish
 // grid (ROW_BLOCKS, l, Z).  out_h[i] = (acc_h[i] - rowfwd(U_h[i])) [P^-1]_{q_i},
-// plus c0 for h = 0 when c0 is given; U column-major, the rest row-major.
-// out0/out1 may alias c0 / the input.
-template <int LOGN>
+// plus c0(X^galois) for h = 0 when c0 is given, or plus the tensor terms d0
+// (h = 0) and d1 (h = 1) of ciphertexts rx, ry ([2][l][N], Z = 1) when rx is
+// given; U column-major, the rest row-major.  out0/out1 may alias c0 only
+// when galois = 1.
+// XF: XF_PLAIN, XF_GATHER (c0 read through X -> X^galois) or XF_MUL (the
+// tensor terms of rx, ry added instead of c0).
+template <int LOGN, int XF>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
-              size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l) {
+              size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 galois, const u32 *rx, const u32 *ry) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -580,9 +843,33 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
         u32 o[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) o[r] = shoup(a[r] - red1(v[r], q) + q, pinv.x, pinv.y, q);
-        if (h == 0 && c0) {
+        if constexpr (XF == XF_MUL) {
+            // relinearisation: + d0 = x0 y0 (h = 0), + d1 = x0 y1 + x1 y0 (h = 1)
+            const size_t lN = (size_t)l * GE::N, li = (size_t)i * GE::N + rowoff;
+            u32 x0[16], y0[16], cc[16];
+            gload<PLAST>(x0, rx + li, lt);
+            gload<PLAST>(y0, ry + li, lt);
+            if (h == 0) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) cc[r] = mulmod(x0[r], y0[r], pk);
+            } else {
+                u32 x1[16], y1[16];
+                gload<PLAST>(x1, rx + lN + li, lt);
+                gload<PLAST>(y1, ry + lN + li, lt);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const u64 d = (u64)x0[r] * y1[r] + (u64)x1[r] * y0[r];
+                    cc[r] = shoup(redc64(d, q, pk.qn, pk.q1s), pk.r32, pk.r32s, q);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) o[r] = red1(o[r] + cc[r], q);
+        } else if (h == 0 && c0) {
             u32 cc[16];
-            gload<PLAST>(cc, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
+            if constexpr (XF == XF_GATHER)
+                load_row_in<PLAST, LOGN, GE::C>(cc, c0 + z * c0z + (size_t)i * GE::N, nullptr, row, lt, galois, pk);
+            else
+                gload<PLAST>(cc, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
 #pragma unroll
             for (int r = 0; r < 16; ++r) o[r] = red1(o[r] + cc[r], q);
         }
@@ -725,6 +1012,12 @@ static size_t colconv_smem(const pc_ctx *c) {
     return sizeof(u32) * (size_t)2 * c->alpha * GE::CPW * GE::COL_LS;
 }
 
+// k_inner with ROT: the packed source columns, 4 words per thread
+template <class GE>
+static constexpr size_t inner_rot_extra() {
+    return sizeof(u32) * 4 * GE::ROW_THREADS;
+}
+
 template <class F>
 static cudaError_t allow_smem(F *f, size_t bytes) {
     return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -736,11 +1029,15 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
         cudaError_t e = allow_smem(k_row<LG, true, false>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_row<LG, false, false>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_row<LG, false, true>, row_smem_bytes<GE>(1));
-        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, row_smem_bytes<GE>(2));
-        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, false>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, true>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, false>, row_smem_bytes<GE>(2));
-        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, false>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_inner_rot<LG, true>, row_smem_bytes<GE>(2) + inner_rot_extra<GE>());
+        if (e == cudaSuccess) e = allow_smem(k_inner_rot<LG, false>, row_smem_bytes<GE>(2) + inner_rot_extra<GE>());
+        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_PLAIN>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_GATHER>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_MUL>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_modup_finish<LG>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_colconv<LG, true>, colconv_smem<GE>(c));
         if (e == cudaSuccess) e = allow_smem(k_colconv<LG, false>, colconv_smem<GE>(c));
@@ -750,20 +1047,21 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
 }
 
 cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
-                       size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s) {
+                       size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s, u32 galois,
+                       const u32 *mul, u32 *xout) {
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, nlimbs, Z);
         if (fwd)
             e = launch_ex(c, k_row<LG, true, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab,
-                          in, out, first_prime, zin, zout, (int)canonical);
+                          in, out, first_prime, zin, zout, (int)canonical, galois, mul, xout);
         else if (cm_out)
             e = launch_ex(c, k_row<LG, false, true>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(1), s, c->tab,
-                          in, out, first_prime, zin, zout, (int)canonical);
+                          in, out, first_prime, zin, zout, (int)canonical, galois, mul, xout);
         else
             e = launch_ex(c, k_row<LG, false, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab,
-                          in, out, first_prime, zin, zout, (int)canonical);
+                          in, out, first_prime, zin, zout, (int)canonical, galois, mul, xout);
     });
     return e;
 }
@@ -803,38 +1101,44 @@ cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t src
 
 cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
                          u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
-                         cudaStream_t s, u32 t0, u32 nt) {
+                         cudaStream_t s, u32 t0, u32 nt, u32 galois, u32 ginv, bool rot) {
+    if (rot && !fused) return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (nt == 0) nt = l + c->alpha - t0;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, nt, Z);
-        const size_t sm = row_smem_bytes<GE>(2);
+        const size_t sm = row_smem_bytes<GE>(2) + (rot ? inner_rot_extra<GE>() : 0);
         const int pi = pintt ? 1 : 0;
-        if (fused && regen)
-            e = launch_ex(c, k_inner<LG, true, true>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z,
-                          acc, accz, l, kp, pi, t0);
-        else if (fused)
-            e = launch_ex(c, k_inner<LG, true, false>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z,
-                          acc, accz, l, kp, pi, t0);
-        else if (regen)
-            e = launch_ex(c, k_inner<LG, false, true>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1,
-                          c1z, acc, accz, l, kp, pi, t0);
-        else
-            e = launch_ex(c, k_inner<LG, false, false>, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1,
-                          c1z, acc, accz, l, kp, pi, t0);
+        auto go = [&](auto kern) {
+            return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z, acc, accz, l,
+                             kp, pi, t0);
+        };
+        auto go_rot = [&](auto kern) {
+            return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z, acc, accz, l,
+                             kp, pi, t0, galois, ginv);
+        };
+        if (rot) e = regen ? go_rot(k_inner_rot<LG, true>) : go_rot(k_inner_rot<LG, false>);
+        else if (fused) e = regen ? go(k_inner<LG, true, true>) : go(k_inner<LG, true, false>);
+        else e = regen ? go(k_inner<LG, false, true>) : go(k_inner<LG, false, false>);
     });
     return e;
 }
 
 cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
-                               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s) {
+                               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s,
+                               u32 galois, const u32 *rx, const u32 *ry) {
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, l, Z);
-        e = launch_ex(c, k_moddown_row<LG>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(2), s, c->tab, U, Uz,
-                      acc, accz, c0, c0z, out0, out1, outz, l);
+        auto go = [&](auto kern) {
+            return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(2), s, c->tab, U, Uz, acc,
+                             accz, c0, c0z, out0, out1, outz, l, galois, rx, ry);
+        };
+        if (rx) e = Z == 1 && ry ? go(k_moddown_row<LG, XF_MUL>) : cudaErrorInvalidValue;
+        else if (galois != 1) e = go(k_moddown_row<LG, XF_GATHER>);
+        else e = go(k_moddown_row<LG, XF_PLAIN>);
     });
     return e;
 }

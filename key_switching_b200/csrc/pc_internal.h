@@ -83,8 +83,12 @@ namespace pc {
 // launchers (kernels.cu); each returns a cudaError_t from the launch.
 // "CM" = column-major limb (element (r, c) at c*R + r), used for the
 // intermediates between row passes and column passes.
+// The inverse pass can read its input limbs through X -> X^galois and / or
+// times the limbs of `mul` (same strides), and store that transformed input
+// (row-major, stride zout) to xout.
 cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
-                       size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s);
+                       size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s, u32 galois = 1,
+                       const u32 *mul = nullptr, u32 *xout = nullptr);
 // scale_mode: 0 none (lazy), 1 N^-1 (canonical)
 cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
                        size_t zin, size_t zout, int scale_mode, cudaStream_t s);
@@ -95,12 +99,17 @@ cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 f
 // out = [2][l][N].  Output CM when out_cm, else row-major.
 cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l,
                            u32 Z, bool out_cm, cudaStream_t s);
-// inner product for target limbs t0 .. t0+nt-1 (nt = 0: through l+alpha-1)
+// inner product for target limbs t0 .. t0+nt-1 (nt = 0: through l+alpha-1).
+// rot (fused only) applies X -> X^galois to the extended limbs (hoisted
+// rotation; ginv = galois^-1 mod 2N).
 cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
                          u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
-                         cudaStream_t s, u32 t0 = 0, u32 nt = 0);
+                         cudaStream_t s, u32 t0 = 0, u32 nt = 0, u32 galois = 1, u32 ginv = 1, bool rot = false);
+// ModDown finish; c0 read through X -> X^galois, or (rx, ry given) the
+// tensor terms d0, d1 of ciphertexts rx, ry added instead of c0.
 cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
-                               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s);
+                               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s,
+                               u32 galois = 1, const u32 *rx = nullptr, const u32 *ry = nullptr);
 cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l, cudaStream_t s);
 cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, cudaStream_t s);
 cudaError_t prepare_kernels(const pc_ctx *c);

@@ -22,7 +22,8 @@ ERRORS = {-1: "PC_E_ARG", -2: "PC_E_ALIGN", -3: "PC_E_CUDA", -4: "PC_E_DEVICE",
 EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_workspace_bytes",
            "pc_set_workspace", "pc_ntt_fwd", "pc_ntt_inv", "pc_modup", "pc_keyswitch_inner",
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
-           "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc")
+           "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc",
+           "pc_rotate", "pc_rotate_hoisted", "pc_relinearize")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
@@ -79,6 +80,12 @@ def lib():
         L.pc_keyswitch.restype = i32
         L.pc_keyswitch_batch.argtypes = [vp, vp, u32, u32, ctypes.POINTER(_Ksk), vp, vp]
         L.pc_keyswitch_batch.restype = i32
+        L.pc_rotate.argtypes = [vp, vp, vp, u32, u32, ctypes.POINTER(_Ksk), vp, vp, vp]
+        L.pc_rotate.restype = i32
+        L.pc_rotate_hoisted.argtypes = [vp, vp, vp, u32, u32, ctypes.POINTER(u32), ctypes.POINTER(_Ksk), vp, vp]
+        L.pc_rotate_hoisted.restype = i32
+        L.pc_relinearize.argtypes = [vp, vp, vp, u32, ctypes.POINTER(_Ksk), vp, vp]
+        L.pc_relinearize.restype = i32
         L.pc_expand_a.argtypes = [vp, ctypes.c_char_p, u32, vp, vp]
         L.pc_expand_a.restype = i32
         L.pc_check.argtypes = [vp]
@@ -245,6 +252,24 @@ class Context:
         arr = (_Ksk * B)(*[k._c() for k in keys])
         _ok(lib().pc_keyswitch_batch(self._h, _ptr(ct), B, l, arr, _ptr(out), _stream(stream)),
             "pc_keyswitch_batch")
+
+    def rotate(self, c0, c1, l: int, galois: int, key: KSK, c0o, c1o, stream=None):
+        k = key._c()
+        _ok(lib().pc_rotate(self._h, _ptr(c0), _ptr(c1), l, galois, ctypes.byref(k), _ptr(c0o), _ptr(c1o),
+                            _stream(stream)), "pc_rotate")
+
+    def rotate_hoisted(self, c0, c1, l: int, galois: Sequence[int], keys: Sequence[KSK], out, stream=None):
+        n = len(galois)
+        assert len(keys) == n
+        gs = (ctypes.c_uint32 * n)(*galois)
+        arr = (_Ksk * n)(*[k._c() for k in keys])
+        _ok(lib().pc_rotate_hoisted(self._h, _ptr(c0), _ptr(c1), l, n, gs, arr, _ptr(out), _stream(stream)),
+            "pc_rotate_hoisted")
+
+    def relinearize(self, x, y, l: int, key: KSK, out, stream=None):
+        k = key._c()
+        _ok(lib().pc_relinearize(self._h, _ptr(x), _ptr(y), l, ctypes.byref(k), _ptr(out), _stream(stream)),
+            "pc_relinearize")
 
     def expand_a(self, seed: bytes, l: int, out, stream=None):
         _ok(lib().pc_expand_a(self._h, bytes(seed), l, _ptr(out), _stream(stream)), "pc_expand_a")

@@ -30,6 +30,8 @@ class Workload:
     key: str             # "square" (s^2 -> s) or "rot" (rotation keys)
     n_ct: int = 1        # ciphertexts per step
     levels: tuple = ()   # () = top level only
+    op: str = "keyswitch"  # "keyswitch", "rotate", "hoisted" (n_rot rotations, one ModUp), "relin"
+    n_rot: int = 1
 
     @property
     def N(self) -> int:
@@ -52,6 +54,13 @@ WORKLOADS = {
     # level sweep at N=2^17, L=40, alpha=5, dnum=8, levels 40..1
     "sweep_n17": Workload("sweep_n17", 17, 40, 5, 31, "hw", "rot",
                           levels=tuple(range(40, 0, -1))),
+    # rotation by one slot (automorphism X -> X^5 fused into the key switch)
+    "rotate_n16": Workload("rotate_n16", 16, 24, 4, 31, "hw", "rot", op="rotate"),
+    # rotations by 1, 2, 4, ..., 128 slots of one ciphertext sharing one ModUp
+    "hoisted8_n16": Workload("hoisted8_n16", 16, 24, 4, 31, "hw", "rot", op="hoisted", n_rot=8),
+    # ciphertext product: tensor, then relinearisation with the s^2 -> s key
+    "relin_mul_n12": Workload("relin_mul_n12", 12, 4, 2, 30, "ternary", "square", op="relin"),
+    "relin_mul_n16": Workload("relin_mul_n16", 16, 24, 4, 31, "hw", "square", op="relin"),
 }
 
 
