@@ -256,7 +256,7 @@ def run_ours(args):
         levels = list(wl.levels) if wl.levels else [L]
         B = wl.n_ct
         nk = wl.n_rot if wl.op == "hoisted" else B  # keys per step
-        ctx.ensure_workspace(max(levels), B)
+        ctx.ensure_workspace(max(levels), max(B, min(wl.n_rot, 16)) if wl.op == "hoisted" else B)
         per_set = (B * (2 * L * N * 4) * (2 if wl.op == "relin" else 1)
                    + nk * wl.dnum * (L + A) * N * 4 * (1 if regen else 2))
         nsets = max(2, math.ceil(2 * L2_BYTES / per_set)) if args.workload != "sweep_n17" else 1

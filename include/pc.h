@@ -194,8 +194,9 @@ int pc_rotate(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, u
  * keys[i] switches s(X^galois[i]) -> s.  out: device [n][2][l][N], rotation i
  * at out + 2 i l N (c0' then c1'), not overlapping c0 or c1.  Results equal
  * the hoisted oracle bit for bit; they differ from pc_rotate's only in the
- * ModUp approximation term, and both decrypt within the same bound.  Needs
- * the workspace for (l, 1). */
+ * ModUp approximation term, and both decrypt within the same bound.  The
+ * rotations run in batches of up to 16 (one set of launches per batch), so
+ * the call needs the workspace for (l, min(n, 16)), else PC_E_WORKSPACE. */
 int pc_rotate_hoisted(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t n,
                       const uint32_t *galois, const pc_ksk *keys, uint32_t *out, pc_stream stream);
 

@@ -513,15 +513,16 @@ int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_str
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
-// How the kernels read a key switch's inputs.  galois != 1: the automorphism
-// X -> X^galois is applied to c1 (ModUp input and own-digit limbs) and c0 as
-// they are read; rot: it is applied to the extended limbs instead (hoisted
-// rotation; ModUp of the unrotated c1 already in the workspace); mul: c1 is
-// the slot-wise product c1 * mul (relinearisation's d2); rx, ry: the tensor
-// terms d0, d1 of ciphertexts rx, ry are added to the outputs instead of c0.
+// How the kernels read a key switch's inputs.  galois != 1 (single
+// rotation): the automorphism X -> X^galois is applied to c1 (ModUp input)
+// and c0 as they are read.  hoist (hoisted rotations): slice z of the batch
+// applies X -> X^hoist[z] to the extended limbs of one shared ModUp output
+// and to c0.  mul: c1 is the slot-wise product c1 * mul (relinearisation's
+// d2); rx, ry: the tensor terms d0, d1 of ciphertexts rx, ry are added to the
+// outputs instead of c0.
 struct KsInput {
-    u32 galois = 1, ginv = 1;
-    bool rot = false;
+    u32 galois = 1;
+    const u32 *hoist = nullptr;
     const u32 *mul = nullptr, *rx = nullptr, *ry = nullptr;
 };
 
@@ -541,36 +542,52 @@ static cudaEvent_t *profile_slot(pc_ctx *c) {
     return nullptr;
 }
 
-// ModUp up to the column-pass output T in the workspace: inverse row pass of
-// c1 (through the input transform), then the conversion kernel.
-static cudaError_t ks_modup(pc_ctx *c, const u32 *c1, size_t cz, u32 l, u32 B, const KsInput &in, cudaStream_t s,
-                            cudaEvent_t *ev) {
-    const Layout Lw = layout(c, l, B);
+// c1 is read transformed by the ModUp row kernel, which then stores that
+// transformed copy in the workspace for the inner product's own-digit limbs
+static bool c1_transformed(const KsInput &in) { return in.galois != 1 || in.mul; }
+
+// ModUp up to the column-pass output T in the workspace (laid out for Blay
+// ciphertexts): inverse row pass of c1 (through the input transform), then
+// the conversion kernel.
+static cudaError_t ks_modup(pc_ctx *c, const u32 *c1, size_t cz, u32 l, u32 B, u32 Blay, const KsInput &in,
+                            cudaStream_t s, cudaEvent_t *ev) {
+    const Layout Lw = layout(c, l, Blay);
     u32 *ws = (u32 *)c->ws;
     auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
     mark(0);
-    const bool xform = (in.galois != 1 && !in.rot) || in.mul;  // c1 is read transformed
-    cudaError_t e = pc::launch_row(c, false, c1, ws + Lw.w1, 0, l, B, cz, Lw.w1z, false, true, s,
-                                   in.rot ? 1u : in.galois, in.mul, xform ? ws + Lw.x : nullptr);
+    cudaError_t e = pc::launch_row(c, false, c1, ws + Lw.w1, 0, l, B, cz, Lw.w1z, false, true, s, in.galois, in.mul,
+                                   c1_transformed(in) ? ws + Lw.x : nullptr);
     mark(1);
     if (e == cudaSuccess) e = pc::launch_colconv(c, 0, ws + Lw.w1, Lw.w1z, ws + Lw.t, Lw.tz, l, B, true, s);
     mark(2);
     return e;
 }
 
-// Inner products, ModDown and the output combination, from T in the workspace.
+// Inner products, ModDown and the output combination of B slices, from T in
+// the workspace (laid out for Blay ciphertexts; one T shared by every slice
+// when hoisting).  Inputs of slice z at stride cz, outputs at stride oz.
 static cudaError_t ks_finish(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u32 l, const pc_ksk *keys, u32 B,
-                             u32 *o0, u32 *o1, const KsInput &in, cudaStream_t s, cudaEvent_t *ev) {
-    const Layout Lw = layout(c, l, B);
+                             u32 Blay, u32 *o0, u32 *o1, size_t oz, const KsInput &in, cudaStream_t s,
+                             cudaEvent_t *ev) {
+    const Layout Lw = layout(c, l, Blay);
     u32 *ws = (u32 *)c->ws;
     u32 *wt = ws + Lw.t, *wacc = ws + Lw.acc, *wu = ws + Lw.u;
+    const size_t tz = in.hoist ? 0 : Lw.tz;
     const bool regen = keys[0].a == nullptr;
     auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
     cudaError_t e = cudaSuccess;
     // own-digit limbs: c1 itself, or the transformed copy ks_modup stored
-    const bool xform = (in.galois != 1 && !in.rot) || in.mul;
-    const u32 *own = xform ? ws + Lw.x : c1;
-    const size_t ownz = xform ? Lw.xz : cz;
+    const u32 *own = c1_transformed(in) ? ws + Lw.x : c1;
+    const size_t ownz = c1_transformed(in) ? Lw.xz : cz;
+    auto rotpack = [&](u32 b0, u32 nb) {
+        pc::RotPack rp{};
+        for (int z = 0; z < pc::KEYS_PER_LAUNCH; ++z) rp.galois[z] = rp.ginv[z] = 1;
+        for (u32 z = 0; z < nb; ++z) {
+            rp.galois[z] = in.hoist ? in.hoist[b0 + z] : in.galois;
+            rp.ginv[z] = inv_mod_2n(rp.galois[z], c->N);
+        }
+        return rp;
+    };
     // The ModDown branch needs only the special-prime accumulators: when not
     // instrumented, those inner products run first on the high-priority
     // internal stream, followed there by the ModDown conversion kernel, while
@@ -586,8 +603,9 @@ static cudaError_t ks_finish(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz,
                 kp.a[i] = keys[b0 + i].a;
                 seed_words(keys[b0 + i].seed, kp.seed[i]);
             }
-            e = pc::launch_inner(c, true, wt + b0 * Lw.tz, Lw.tz, own + b0 * ownz, ownz, wacc + b0 * Lw.accz,
-                                 Lw.accz, l, kp, nb, regen, true, st, t0, nt, in.galois, in.ginv, in.rot);
+            const pc::RotPack rp = rotpack(b0, nb);
+            e = pc::launch_inner(c, true, wt + b0 * tz, tz, own + b0 * ownz, ownz, wacc + b0 * Lw.accz, Lw.accz, l,
+                                 kp, nb, regen, true, st, t0, nt, in.hoist ? &rp : nullptr);
         }
     };
     if (fork) {
@@ -604,9 +622,12 @@ static cudaError_t ks_finish(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz,
         if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, Lw.accz, wu, Lw.uz, l, B, true, s);
     }
     mark(4);
+    const bool rot = in.hoist || in.galois != 1;
+    if (rot && B > (u32)pc::KEYS_PER_LAUNCH) e = cudaErrorInvalidValue;
+    const pc::RotPack rp = rotpack(0, B < (u32)pc::KEYS_PER_LAUNCH ? B : (u32)pc::KEYS_PER_LAUNCH);
     if (e == cudaSuccess)
-        e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, in.rx ? nullptr : c0, cz, o0, o1, cz, l, B, s,
-                                   in.galois, in.rx, in.ry);
+        e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, in.rx ? nullptr : c0, cz, o0, o1, oz, l, B, s,
+                                   rot ? &rp : nullptr, in.rx, in.ry);
     mark(5);
     return e;
 }
@@ -619,8 +640,8 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
     for (u32 b = 1; b < B; ++b)
         if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
     cudaEvent_t *ev = profile_slot(c);
-    cudaError_t e = ks_modup(c, c1, cz, l, B, in, s, ev);
-    if (e == cudaSuccess) e = ks_finish(c, c0, c1, cz, l, keys, B, o0, o1, in, s, ev);
+    cudaError_t e = ks_modup(c, c1, cz, l, B, B, in, s, ev);
+    if (e == cudaSuccess) e = ks_finish(c, c0, c1, cz, l, keys, B, B, o0, o1, cz, in, s, ev);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
@@ -679,18 +700,18 @@ int pc_rotate_hoisted(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_
     if (!aligned16(c0) || !aligned16(c1) || !aligned16(out)) return PC_E_ALIGN;
     const size_t lN = (size_t)l * c->N, ob = 2 * (size_t)n * lN * sizeof(u32);
     if (overlaps(out, ob, c0, lN * sizeof(u32)) || overlaps(out, ob, c1, lN * sizeof(u32))) return PC_E_ARG;
-    if (int r = need_ws(c, l, 1)) return r;
+    // slices of up to KEYS_PER_LAUNCH rotations share one ModUp output
+    const u32 Blay = n < (u32)pc::KEYS_PER_LAUNCH ? n : (u32)pc::KEYS_PER_LAUNCH;
+    if (int r = need_ws(c, l, Blay)) return r;
     DeviceGuard dg(c->device);
     const cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = ks_modup(c, c1, 0, l, 1, KsInput{}, s, nullptr);
-    for (u32 i = 0; e == cudaSuccess && i < n; ++i) {
+    cudaError_t e = ks_modup(c, c1, 0, l, 1, Blay, KsInput{}, s, nullptr);
+    for (u32 i0 = 0; e == cudaSuccess && i0 < n; i0 += Blay) {
+        const u32 nb = n - i0 < Blay ? n - i0 : Blay;
         KsInput in;
-        in.galois = galois[i];
-        in.ginv = inv_mod_2n(galois[i], c->N);
-        if (((in.galois * in.ginv) & (2u * c->N - 1u)) != 1u) return PC_E_ARG;  // cannot happen for odd g
-        in.rot = true;
-        u32 *o = out + 2 * (size_t)i * lN;
-        e = ks_finish(c, c0, c1, 0, l, &keys[i], 1, o, o + lN, in, s, nullptr);
+        in.hoist = galois + i0;
+        u32 *o = out + 2 * (size_t)i0 * lN;
+        e = ks_finish(c, c0, c1, 0, l, keys + i0, nb, Blay, o, o + lN, 2 * lN, in, s, nullptr);
     }
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }

@@ -789,25 +789,34 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
     }
 }
 
+// element z of a parameter array without copying the array to local memory
+__device__ __forceinline__ u32 pick(const u32 (&a)[KEYS_PER_LAUNCH], u32 z) {
+    u32 v = a[0];
+#pragma unroll
+    for (int i = 1; i < KEYS_PER_LAUNCH; ++i) v = (z == (u32)i) ? a[i] : v;
+    return v;
+}
+
 template <int LOGN, bool REGEN>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 4)
 k_inner_rot(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
-            KeyPack kp, int pintt, u32 t0, u32 galois, u32 ginv) {
-    inner_body<LOGN, true, REGEN, true>(T, src, srcz, c1, c1z, acc, accz, l, kp, pintt, t0, galois, ginv);
+            KeyPack kp, int pintt, u32 t0, RotPack rp) {
+    inner_body<LOGN, true, REGEN, true>(T, src, srcz, c1, c1z, acc, accz, l, kp, pintt, t0,
+                                        pick(rp.galois, blockIdx.z), pick(rp.ginv, blockIdx.z));
 }
 
 // ----------------------------------------------------------- ModDown finish
 // grid (ROW_BLOCKS, l, Z).  out_h[i] = (acc_h[i] - rowfwd(U_h[i])) [P^-1]_{q_i},
-// plus c0(X^galois) for h = 0 when c0 is given, or plus the tensor terms d0
-// (h = 0) and d1 (h = 1) of ciphertexts rx, ry ([2][l][N], Z = 1) when rx is
-// given; U column-major, the rest row-major.  out0/out1 may alias c0 only
-// when galois = 1.
-// XF: XF_PLAIN, XF_GATHER (c0 read through X -> X^galois) or XF_MUL (the
-// tensor terms of rx, ry added instead of c0).
+// plus c0 for h = 0 when c0 is given, or plus the tensor terms d0 (h = 0)
+// and d1 (h = 1) of ciphertexts rx, ry ([2][l][N], Z = 1) when rx is given;
+// U column-major, the rest row-major.  out0/out1 may alias c0 only for
+// XF_PLAIN.
+// XF: XF_PLAIN, XF_GATHER (c0 of slice z read through X -> X^rp.galois[z])
+// or XF_MUL (the tensor terms of rx, ry added instead of c0).
 template <int LOGN, int XF>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
-              size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 galois, const u32 *rx, const u32 *ry) {
+              size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, RotPack rp, const u32 *rx, const u32 *ry) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -867,7 +876,8 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
         } else if (h == 0 && c0) {
             u32 cc[16];
             if constexpr (XF == XF_GATHER)
-                load_row_in<PLAST, LOGN, GE::C>(cc, c0 + z * c0z + (size_t)i * GE::N, nullptr, row, lt, galois, pk);
+                load_row_in<PLAST, LOGN, GE::C>(cc, c0 + z * c0z + (size_t)i * GE::N, nullptr, row, lt,
+                                                pick(rp.galois, z), pk);
             else
                 gload<PLAST>(cc, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
 #pragma unroll
@@ -1101,8 +1111,8 @@ cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t src
 
 cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
                          u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
-                         cudaStream_t s, u32 t0, u32 nt, u32 galois, u32 ginv, bool rot) {
-    if (rot && !fused) return cudaErrorInvalidValue;
+                         cudaStream_t s, u32 t0, u32 nt, const RotPack *rot) {
+    if (rot && (!fused || Z > (u32)KEYS_PER_LAUNCH)) return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (nt == 0) nt = l + c->alpha - t0;
     PC_DISPATCH(c->logN, {
@@ -1116,7 +1126,7 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
         };
         auto go_rot = [&](auto kern) {
             return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z, acc, accz, l,
-                             kp, pi, t0, galois, ginv);
+                             kp, pi, t0, *rot);
         };
         if (rot) e = regen ? go_rot(k_inner_rot<LG, true>) : go_rot(k_inner_rot<LG, false>);
         else if (fused) e = regen ? go(k_inner<LG, true, true>) : go(k_inner<LG, true, false>);
@@ -1127,17 +1137,21 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
 
 cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
                                size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s,
-                               u32 galois, const u32 *rx, const u32 *ry) {
+                               const RotPack *rot, const u32 *rx, const u32 *ry) {
+    if (rot && Z > (u32)KEYS_PER_LAUNCH) return cudaErrorInvalidValue;
+    RotPack rp{};
+    for (int z = 0; z < KEYS_PER_LAUNCH; ++z) rp.galois[z] = rp.ginv[z] = 1;
+    if (rot) rp = *rot;
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, l, Z);
         auto go = [&](auto kern) {
             return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(2), s, c->tab, U, Uz, acc,
-                             accz, c0, c0z, out0, out1, outz, l, galois, rx, ry);
+                             accz, c0, c0z, out0, out1, outz, l, rp, rx, ry);
         };
         if (rx) e = Z == 1 && ry ? go(k_moddown_row<LG, XF_MUL>) : cudaErrorInvalidValue;
-        else if (galois != 1) e = go(k_moddown_row<LG, XF_GATHER>);
+        else if (rot) e = go(k_moddown_row<LG, XF_GATHER>);
         else e = go(k_moddown_row<LG, XF_PLAIN>);
     });
     return e;

@@ -50,6 +50,13 @@ struct KeyPack {
     u32 seed[KEYS_PER_LAUNCH][8];
 };
 
+// Automorphism X -> X^galois[z] (and galois[z]^-1 mod 2N) for grid slice z
+// of a rotation launch, by value in the kernel parameters; 1 = none.
+struct RotPack {
+    u32 galois[KEYS_PER_LAUNCH];
+    u32 ginv[KEYS_PER_LAUNCH];
+};
+
 }  // namespace pc
 
 struct pc_ctx {
@@ -100,16 +107,17 @@ cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 f
 cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l,
                            u32 Z, bool out_cm, cudaStream_t s);
 // inner product for target limbs t0 .. t0+nt-1 (nt = 0: through l+alpha-1).
-// rot (fused only) applies X -> X^galois to the extended limbs (hoisted
-// rotation; ginv = galois^-1 mod 2N).
+// rot (fused only) applies X -> X^galois[z] to the extended limbs of slice z
+// (hoisted rotations).
 cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
                          u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
-                         cudaStream_t s, u32 t0 = 0, u32 nt = 0, u32 galois = 1, u32 ginv = 1, bool rot = false);
-// ModDown finish; c0 read through X -> X^galois, or (rx, ry given) the
-// tensor terms d0, d1 of ciphertexts rx, ry added instead of c0.
+                         cudaStream_t s, u32 t0 = 0, u32 nt = 0, const RotPack *rot = nullptr);
+// ModDown finish; c0 of slice z read through X -> X^galois[z] when rot is
+// given, or (rx, ry given) the tensor terms d0, d1 of ciphertexts rx, ry
+// added instead of c0.
 cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
                                size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s,
-                               u32 galois = 1, const u32 *rx = nullptr, const u32 *ry = nullptr);
+                               const RotPack *rot = nullptr, const u32 *rx = nullptr, const u32 *ry = nullptr);
 cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l, cudaStream_t s);
 cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, cudaStream_t s);
 cudaError_t prepare_kernels(const pc_ctx *c);

@@ -63,7 +63,7 @@ def test_rotate_hoisted(built, oracle, logN, L, alpha, bits):
     keys = [G.random_key(P, 200 + i) for i in range(len(gs))]
     kk = [pc.KSK(s, G.dev(b)) for s, b in keys]
     for l in sorted({L, alpha + 1, 1}, reverse=True):
-        C.ensure_workspace(l)
+        C.ensure_workspace(l, len(gs))
         c0, c1 = _ct(P, l, 60 + l)
         out = G.filled(len(gs), 2, l, P.N)
         C.rotate_hoisted(G.dev(c0), G.dev(c1), l, gs, kk, out)
@@ -137,7 +137,7 @@ def test_rotate_hoisted_n16_full_size(built, oracle):
     from key_switching_b200 import pc
     P, C = G.contexts(oracle, 16, 24, 4, 31)
     l = 24
-    C.ensure_workspace(l)
+    C.ensure_workspace(l, 4)
     gs = [oracle.galois_elt(r, 16) for r in (1, 2, 4, 8)]
     keys = [G.random_key(P, 300 + i) for i in range(4)]
     kk = [pc.KSK(s, G.dev(b)) for s, b in keys]
@@ -207,6 +207,10 @@ def test_rotation_error_paths(built, oracle):
     with pytest.raises(pc.PCError) as ei:
         C.rotate_hoisted(c0, c1, 4, [5, 6], [key, key], out)
     assert ei.value.code == -1
+    with pytest.raises(pc.PCError) as ei:  # two rotations need two slices of workspace
+        C.rotate_hoisted(c0, c1, 4, [5, 25], [key, key], out)
+    assert ei.value.code == -7
+    C.ensure_workspace(4, 2)
     x = G.empty(2, 4, P.N)
     with pytest.raises(pc.PCError) as ei:
         C.relinearize(x, x, 4, key, x)
