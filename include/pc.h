@@ -171,6 +171,23 @@ int pc_keyswitch(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l
 int pc_keyswitch_batch(pc_ctx *ctx, const uint32_t *ct, uint32_t B, uint32_t l,
                        const pc_ksk *keys, uint32_t *out, pc_stream stream);
 
+/* Key switches of n ciphertexts held in HOST memory: ct and out are host
+ * arrays [n][2][l][N] (c0 then c1 of each ciphertext, natural layout as in
+ * device calls); keys: host array of n keys (device 'b' halves, as in
+ * pc_keyswitch).  The library pipelines them through two device staging
+ * slots: while ciphertext k is key-switched on `stream`, ciphertext k+1 is
+ * copied in and ciphertext k-1 copied out on two internal streams, so copies
+ * and kernels overlap (with page-locked host buffers; pageable ones work but
+ * copy synchronously).  One cudaMemcpyAsync per ciphertext and direction.
+ * Asynchronous: `stream` completes after the last output has reached the
+ * host.  out must not overlap ct.  Needs a workspace of
+ * pc_host_workspace_bytes(l) (the key switch's plus the staging slots), else
+ * PC_E_WORKSPACE.  The pages have no counterpart of this call: it is the
+ * host-facing entry point of the same key switch. */
+size_t pc_host_workspace_bytes(const pc_ctx *ctx, uint32_t l);
+int pc_keyswitch_host(pc_ctx *ctx, const uint32_t *ct, uint32_t n, uint32_t l, const pc_ksk *keys,
+                      uint32_t *out, pc_stream stream);
+
 /* Rotation: the key switch of c(X^g) = (c0(X^g), c1(X^g)) -- the ciphertext
  * under the automorphism X -> X^g, which decrypts under s(X^g) -- with a key
  * k for s(X^g) -> s.  (Perseus README, "Python API": the session holds keys

@@ -387,6 +387,14 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
         e = cudaStreamCreateWithPriority(&c->aux, cudaStreamNonBlocking, hi_pri);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->h2d, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->d2h, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming);
+        for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&c->ev_in[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_done[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_out[i], cudaEventDisableTiming);
+        }
         if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
         c->overlap = getenv("PC_NO_OVERLAP") ? 0 : 1;
     }
@@ -419,6 +427,11 @@ void pc_ctx_destroy(pc_ctx *c) {
     if (c->aux) cudaStreamDestroy(c->aux);
     if (c->ev_fork) cudaEventDestroy(c->ev_fork);
     if (c->ev_join) cudaEventDestroy(c->ev_join);
+    if (c->h2d) cudaStreamDestroy(c->h2d);
+    if (c->d2h) cudaStreamDestroy(c->d2h);
+    for (cudaEvent_t ev : {c->ev_start, c->ev_in[0], c->ev_in[1], c->ev_done[0], c->ev_done[1], c->ev_out[0],
+                           c->ev_out[1]})
+        if (ev) cudaEventDestroy(ev);
     if (c->dev_block) cudaFree(c->dev_block);
     delete c;
 }
@@ -428,6 +441,15 @@ uint32_t pc_psi(const pc_ctx *c, uint32_t g) { return (c && g < c->NP) ? c->psi[
 size_t pc_workspace_bytes(const pc_ctx *c, uint32_t l, uint32_t B) {
     if (!c || l < 1 || l > c->L || B < 1) return 0;
     return layout(c, l, B).total * sizeof(u32);
+}
+
+// pc_keyswitch_host: the key switch's workspace, then two staging slots of
+// one ciphertext in and one out ([2][l][N] each)
+static size_t host_ws_words(const pc_ctx *c, u32 l) { return layout(c, l, 1).total + 8 * (size_t)l * c->N; }
+
+size_t pc_host_workspace_bytes(const pc_ctx *c, uint32_t l) {
+    if (!c || l < 1 || l > c->L) return 0;
+    return host_ws_words(c, l) * sizeof(u32);
 }
 
 int pc_set_workspace(pc_ctx *c, void *dev, size_t bytes) {
@@ -732,6 +754,49 @@ int pc_relinearize(pc_ctx *c, const uint32_t *x, const uint32_t *y, uint32_t l, 
     in.rx = x;
     in.ry = y;
     return keyswitch_core(c, nullptr, x + lN, 0, l, k, 1, out, out + lN, (cudaStream_t)stream, in);
+}
+
+int pc_keyswitch_host(pc_ctx *c, const uint32_t *ct, uint32_t n, uint32_t l, const pc_ksk *keys, uint32_t *out,
+                      pc_stream stream) {
+    if (!c || !ct || !out || !keys || n < 1 || l < 1 || l > c->L) return PC_E_ARG;
+    for (u32 k = 0; k < n; ++k)
+        if (int r = check_ksk(c, &keys[k])) return r;
+    const size_t lN = (size_t)l * c->N, cb = 2 * lN * sizeof(u32);
+    if (overlaps(ct, n * cb, out, n * cb)) return PC_E_ARG;
+    if (!c->ws || c->ws_bytes < host_ws_words(c, l) * sizeof(u32)) return PC_E_WORKSPACE;
+    DeviceGuard dg(c->device);
+    const cudaStream_t s = (cudaStream_t)stream;
+    u32 *stage = (u32 *)c->ws + layout(c, l, 1).total;
+    u32 *din[2] = {stage, stage + 4 * lN}, *dout[2] = {stage + 2 * lN, stage + 6 * lN};
+    // the copy streams start after the work already queued on `stream`
+    cudaError_t e = cudaEventRecord(c->ev_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(c->h2d, c->ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(c->d2h, c->ev_start, 0);
+    int rc = e == cudaSuccess ? PC_OK : cuda_fail(e);
+    for (u32 k = 0; rc == PC_OK && k < n; ++k) {
+        const int i = k & 1;
+        // slot i is free for input once key switch k-2 is done with it
+        if (k >= 2) e = cudaStreamWaitEvent(c->h2d, c->ev_done[i], 0);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(din[i], ct + k * 2 * lN, cb, cudaMemcpyHostToDevice, c->h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(c->ev_in[i], c->h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, c->ev_in[i], 0);
+        // and free for output once copy k-2 has left it
+        if (e == cudaSuccess && k >= 2) e = cudaStreamWaitEvent(s, c->ev_out[i], 0);
+        if (e != cudaSuccess) { rc = cuda_fail(e); break; }
+        rc = keyswitch_core(c, din[i], din[i] + lN, 0, l, &keys[k], 1, dout[i], dout[i] + lN, s);
+        if (rc != PC_OK) break;
+        e = cudaEventRecord(c->ev_done[i], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(c->d2h, c->ev_done[i], 0);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(out + k * 2 * lN, dout[i], cb, cudaMemcpyDeviceToHost, c->d2h);
+        if (e == cudaSuccess) e = cudaEventRecord(c->ev_out[i], c->d2h);
+        if (e != cudaSuccess) rc = cuda_fail(e);
+    }
+    // `stream` completes only after every output has reached the host
+    for (u32 k = n >= 2 ? n - 2 : 0; k < n; ++k) {
+        const cudaError_t w = cudaStreamWaitEvent(s, c->ev_out[k & 1], 0);
+        if (rc == PC_OK && w != cudaSuccess) rc = cuda_fail(w);
+    }
+    return rc;
 }
 
 int pc_expand_a(pc_ctx *c, const uint8_t seed[32], uint32_t l, uint32_t *a_out, pc_stream stream) {

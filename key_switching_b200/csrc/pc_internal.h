@@ -80,6 +80,10 @@ struct pc_ctx {
     int overlap;
     cudaStream_t aux;
     cudaEvent_t ev_fork, ev_join;
+    // host-buffer pipeline (pc_keyswitch_host): copy streams and, per staging
+    // slot, "input landed", "key switch done" and "output copied" events
+    cudaStream_t h2d, d2h;
+    cudaEvent_t ev_start, ev_in[2], ev_done[2], ev_out[2];
     // per-kernel timing (pc_profile_begin / pc_profile_end)
     cudaEvent_t *prof_ev;   // [prof_max][PC_PROFILE_STAGES + 1]
     uint32_t prof_max, prof_used, prof_every, prof_seen;

@@ -23,7 +23,7 @@ EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_wor
            "pc_set_workspace", "pc_ntt_fwd", "pc_ntt_inv", "pc_modup", "pc_keyswitch_inner",
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
            "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc",
-           "pc_rotate", "pc_rotate_hoisted", "pc_relinearize")
+           "pc_rotate", "pc_rotate_hoisted", "pc_relinearize", "pc_keyswitch_host", "pc_host_workspace_bytes")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
@@ -86,6 +86,10 @@ def lib():
         L.pc_rotate_hoisted.restype = i32
         L.pc_relinearize.argtypes = [vp, vp, vp, u32, ctypes.POINTER(_Ksk), vp, vp]
         L.pc_relinearize.restype = i32
+        L.pc_keyswitch_host.argtypes = [vp, vp, u32, u32, ctypes.POINTER(_Ksk), vp, vp]
+        L.pc_keyswitch_host.restype = i32
+        L.pc_host_workspace_bytes.argtypes = [vp, u32]
+        L.pc_host_workspace_bytes.restype = sz
         L.pc_expand_a.argtypes = [vp, ctypes.c_char_p, u32, vp, vp]
         L.pc_expand_a.restype = i32
         L.pc_check.argtypes = [vp]
@@ -121,6 +125,15 @@ def _ptr(t) -> int:
         return t
     assert t.is_cuda and t.is_contiguous() and t.element_size() == 4, "need a contiguous 32-bit CUDA tensor"
     return t.data_ptr()
+
+
+def _hptr(a) -> int:
+    """Host address of a contiguous 4-byte-element CPU torch tensor or numpy array."""
+    if hasattr(a, "is_cuda"):
+        assert not a.is_cuda and a.is_contiguous() and a.element_size() == 4, "need a contiguous 32-bit CPU tensor"
+        return a.data_ptr()
+    assert a.flags["C_CONTIGUOUS"] and a.itemsize == 4, "need a contiguous 32-bit array"
+    return a.ctypes.data
 
 
 def _stream(stream) -> Optional[int]:
@@ -265,6 +278,24 @@ class Context:
         arr = (_Ksk * n)(*[k._c() for k in keys])
         _ok(lib().pc_rotate_hoisted(self._h, _ptr(c0), _ptr(c1), l, n, gs, arr, _ptr(out), _stream(stream)),
             "pc_rotate_hoisted")
+
+    def host_workspace_bytes(self, l: int) -> int:
+        return lib().pc_host_workspace_bytes(self._h, l)
+
+    def ensure_host_workspace(self, l: int):
+        """Allocate (with torch) and set a workspace big enough for keyswitch_host at level l."""
+        import torch
+        need = self.host_workspace_bytes(l)
+        if self._ws is None or self._ws.numel() * self._ws.element_size() < need:
+            self.set_workspace(torch.empty(need, dtype=torch.uint8, device=f"cuda:{self.device}"))
+        return self._ws
+
+    def keyswitch_host(self, ct, n: int, l: int, keys: Sequence[KSK], out, stream=None):
+        """n key switches of host ciphertexts ct [n][2][l][N] into host out [n][2][l][N]."""
+        assert len(keys) == n
+        arr = (_Ksk * n)(*[k._c() for k in keys])
+        _ok(lib().pc_keyswitch_host(self._h, _hptr(ct), n, l, arr, _hptr(out), _stream(stream)),
+            "pc_keyswitch_host")
 
     def relinearize(self, x, y, l: int, key: KSK, out, stream=None):
         k = key._c()
