@@ -215,6 +215,27 @@ def test_batch16_n16(built, oracle):
         assert np.array_equal(got[k, 0], G.host(o0)) and np.array_equal(got[k, 1], G.host(o1)), k
 
 
+def test_batch_more_than_one_launch(built, oracle):
+    """20 ciphertexts with 20 keys: the inner product runs in two launches of
+    16 + 4 keys; every ciphertext bit-exact with the oracle (small ring)."""
+    from key_switching_b200 import pc
+    P, C = G.contexts(oracle, 11, 7, 3, 31)
+    l, B = 6, 20
+    C.ensure_workspace(l, B)
+    keys, bs = [], []
+    for k in range(B):
+        seed, b = G.random_key(P, 700 + k)
+        bs.append(b)
+        keys.append(pc.KSK(seed, G.dev(b)))
+    ct = np.stack([np.stack([synth.uniform_residues(P.q[:l], P.N, 8, k, h) for h in range(2)]) for k in range(B)])
+    out = G.filled(B, 2, l, P.N)
+    C.keyswitch_batch(G.dev(ct), B, l, keys, out)
+    got = G.host(out)
+    for k in range(B):
+        w0, w1 = oracle.keyswitch(P, ct[k, 0], ct[k, 1], l, keys[k].seed, bs[k])
+        assert np.array_equal(got[k, 0], w0) and np.array_equal(got[k, 1], w1), k
+
+
 @pytest.mark.parametrize("l", [40, 23, 6, 1])
 def test_sweep_n17_levels(built, oracle, l):
     """N=2^17, L=40, alpha=5, dnum=8 at sampled levels of the 40..1 sweep."""

@@ -75,6 +75,50 @@ def test_rotate_hoisted(built, oracle, logN, L, alpha, bits):
     C.check()
 
 
+def test_rotate_hoisted_more_than_one_batch(built, oracle):
+    """18 hoisted rotations: two launch batches (16 + 2) over one ModUp, each
+    rotation bit-exact with the oracle, l below L."""
+    from key_switching_b200 import pc
+    P, C = G.contexts(oracle, 10, 5, 2, 30)
+    N = P.N
+    gs = [pow(5, r, 2 * N) for r in range(1, 19)]
+    keys = [G.random_key(P, 600 + i) for i in range(len(gs))]
+    kk = [pc.KSK(s, G.dev(b)) for s, b in keys]
+    l = 4
+    C.ensure_workspace(l, 16)
+    c0, c1 = _ct(P, l, 70)
+    out = G.filled(len(gs), 2, l, N)
+    C.rotate_hoisted(G.dev(c0), G.dev(c1), l, gs, kk, out)
+    got = G.host(out)
+    want = oracle.rotate_hoisted(P, c0, c1, l, gs, [s for s, _ in keys], [b for _, b in keys])
+    for i, (w0, w1) in enumerate(want):
+        assert np.array_equal(got[i, 0], w0) and np.array_equal(got[i, 1], w1), i
+    C.check()
+
+
+def test_rotate_n17_low_level(built, oracle):
+    """N=2^17, L=40, alpha=5 (the level-sweep basis) at l=7: a single and two
+    hoisted rotations, bit-exact."""
+    from key_switching_b200 import pc
+    P, C = G.contexts(oracle, 17, 40, 5, 31)
+    l = 7
+    C.ensure_workspace(l, 2)
+    seed, b = G.random_key(P, 17)
+    key = pc.KSK(seed, G.dev(b))
+    c0, c1 = _ct(P, l, 80)
+    g = oracle.galois_elt(3, 17)
+    o0, o1 = G.filled(l, P.N), G.filled(l, P.N)
+    C.rotate(G.dev(c0), G.dev(c1), l, g, key, o0, o1)
+    w0, w1 = oracle.rotate(P, c0, c1, l, g, seed, b)
+    assert np.array_equal(G.host(o0), w0) and np.array_equal(G.host(o1), w1)
+    gs = [g, 2 * P.N - 1]
+    out = G.filled(2, 2, l, P.N)
+    C.rotate_hoisted(G.dev(c0), G.dev(c1), l, gs, [key, key], out)
+    got = G.host(out)
+    for i, (h0, h1) in enumerate(oracle.rotate_hoisted(P, c0, c1, l, gs, [seed, seed], [b, b])):
+        assert np.array_equal(got[i, 0], h0) and np.array_equal(got[i, 1], h1), i
+
+
 @pytest.mark.parametrize("logN,L,alpha,bits", SMALL)
 def test_relinearize(built, oracle, logN, L, alpha, bits):
     from key_switching_b200 import pc
