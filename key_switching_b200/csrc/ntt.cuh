@@ -44,7 +44,7 @@ struct Phase {
     }
 
     // forward stages; tw(s, u, hi, b) returns {w, w'} for the table entry
-    // (1 << s) + (hi << u) + b of stage s = S0 + u (see TwNatural / TwRowSm)
+    // (1 << s) + (hi << u) + b of stage s = S0 + u (natural layout; see TwRow for the stored one)
     template <class TW>
     __device__ static __forceinline__ void fwd(u32 v[16], int lt, const TW &tw, u32 q) {
 #pragma unroll
@@ -105,20 +105,12 @@ struct Plan {
 };
 
 // Barriers that order a line's shared-memory exchange: a warp barrier when
-// every line's threads sit in one warp (row passes), a CTA barrier, or a
-// named barrier shared by one group of `n` threads (column passes run by
-// independent thread groups).
+// every line's threads sit in one warp, else a CTA barrier.
 struct SyncWarp {
     __device__ __forceinline__ void operator()() const { __syncwarp(); }
 };
 struct SyncCta {
     __device__ __forceinline__ void operator()() const { __syncthreads(); }
-};
-struct SyncGroup {
-    int id, n;  // barrier id (1..15) and thread count (a multiple of 32)
-    __device__ __forceinline__ void operator()() const {
-        asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
-    }
 };
 
 // Exchange the registers of phase A's layout into phase B's layout through
@@ -131,23 +123,6 @@ __device__ __forceinline__ void exchange(u32 v[16], u32 *sm, int lt, const ADDR 
     sync();
 #pragma unroll
     for (int r = 0; r < 16; ++r) v[r] = sm[addr(PB::x_of(lt, r))];
-}
-
-template <class PA, class PB, class SYNC, class ADDR>
-__device__ __forceinline__ void exchange2(u32 v0[16], u32 v1[16], u32 *sm0, u32 *sm1, int lt, const ADDR &addr,
-                                          const SYNC &sync) {
-    sync();
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        sm0[addr(PA::x_of(lt, r))] = v0[r];
-        sm1[addr(PA::x_of(lt, r))] = v1[r];
-    }
-    sync();
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        v0[r] = sm0[addr(PB::x_of(lt, r))];
-        v1[r] = sm1[addr(PB::x_of(lt, r))];
-    }
 }
 
 // Full forward line transform: registers enter at Plan::fwd_in positions and
@@ -164,27 +139,6 @@ __device__ __forceinline__ void line_fwd(u32 v[16], u32 *sm, int lt, const ADDR 
     if constexpr (PL::NPH >= 3) {
         exchange<typename PL::P1, typename PL::P2>(v, sm, lt, addr, sync);
         PL::P2::fwd(v, lt, tw, q);
-    }
-}
-
-// Two independent forward line transforms advanced together (separate
-// primes, twiddle tables and exchange lines): twice the independent work
-// between the shared barriers.
-template <int LOGM, class ADDR, class TW0, class TW1, class SYNC>
-__device__ __forceinline__ void line_fwd2(u32 v0[16], u32 v1[16], u32 *sm0, u32 *sm1, int lt, const ADDR &addr,
-                                          const TW0 &tw0, const TW1 &tw1, u32 q0, u32 q1, const SYNC &sync) {
-    using PL = Plan<LOGM>;
-    PL::P0::fwd(v0, lt, tw0, q0);
-    PL::P0::fwd(v1, lt, tw1, q1);
-    if constexpr (PL::NPH >= 2) {
-        exchange2<typename PL::P0, typename PL::P1>(v0, v1, sm0, sm1, lt, addr, sync);
-        PL::P1::fwd(v0, lt, tw0, q0);
-        PL::P1::fwd(v1, lt, tw1, q1);
-    }
-    if constexpr (PL::NPH >= 3) {
-        exchange2<typename PL::P1, typename PL::P2>(v0, v1, sm0, sm1, lt, addr, sync);
-        PL::P2::fwd(v0, lt, tw0, q0);
-        PL::P2::fwd(v1, lt, tw1, q1);
     }
 }
 
@@ -205,13 +159,6 @@ __device__ __forceinline__ void line_inv(u32 v[16], u32 *sm, int lt, const ADDR 
     PL::P0::inv(v, lt, tw, q);
 }
 
-// Twiddle tables.  Natural layout: entry (1 << s) + (hi << u) + b.
-struct TwNatural {
-    const uint2 *t;
-    __device__ __forceinline__ uint2 operator()(int s, int u, int hi, int b) const {
-        return t[(1 << s) + (hi << u) + b];
-    }
-};
 // Twiddle tables as stored on the device ("re-laid"): within stage s, with
 // u = s mod 4 and S0 = s - u (the first stage of its radix-16 phase), the
 // natural entry (1 << s) + (hi << u) + b sits at (1 << s) + (b << S0) + hi.
