@@ -158,3 +158,23 @@ def test_decrypt_after_relinearisation(oracle, logN, L, alpha, bits):
         Ql = H.prod(P.q[:l])
         err = max(abs(int(v)) for v in H.centered(H.crt_lift(np.stack(diffs), P.q[:l]), Ql))
         assert err <= _bound(P, l, s, e) < Ql // 2, (l, err)
+
+
+@pytest.mark.parametrize("logN", [10, 12, 16, 17])
+def test_automorphism_maps_row_blocks_to_row_blocks(oracle, logN):
+    """The property the GPU rotation kernels are built on, derived from the
+    oracle's own automorphism: in the R x C view of a limb (C = 2^min(8,
+    logN-4) words per row) X -> X^g takes every row to a single row and every
+    aligned block of 8 rows onto an aligned block of 8 rows."""
+    N = 1 << logN
+    C = 1 << min(8, logN - 4)
+    R = N // C
+    idx = np.arange(N, dtype=np.uint32)
+    for g in sorted({5, oracle.galois_elt(N // 2 - 1, logN), 2 * N - 1, oracle.galois_elt(3, logN) * (2 * N - 1) % (2 * N)}):
+        src = oracle.automorph_ntt(idx, logN, g).astype(np.int64)  # slot k of x(X^g) is slot src[k] of x
+        rows = (src // C).reshape(R, C)
+        assert (rows == rows[:, :1]).all(), g                   # one source row per output row
+        rho = rows[:, 0]
+        assert sorted(rho.tolist()) == list(range(R)), g          # a permutation of the rows
+        blocks = rho.reshape(R // 8, 8)
+        assert (blocks // 8 == blocks[:, :1] // 8).all(), g       # aligned 8-blocks onto aligned 8-blocks
