@@ -421,7 +421,8 @@ def run_ours(args):
         res["e2e"] = {"value": whole_job_rate(1, ke, world, ems), "unit": unit,
                       "h2d_bytes_per_step": 2 * l * N * 4, "d2h_bytes_per_step": 2 * l * N * 4}
 
-    if rank == 0 and not args.no_cpu_baseline and args.workload in ("rot1_n16", "relin_n12"):
+    # the oracle's CPU baseline: rank 0 of a single-GPU run only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in ("rot1_n16", "relin_n12"):
         res["cpu_baseline"] = cpu_baseline(wl, q, p, budget_s=args.cpu_budget)
 
     if dist:
