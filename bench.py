@@ -227,6 +227,8 @@ def run_ours(args):
         return pc.KSK(synth.chacha_seed(seed_id, rank), dev(b), a)
 
     launches_per_step = 5
+    graphs = None
+    PROF_EVERY = 10  # sampled steps carry per-kernel events; the rest run uninstrumented
     if args.workload == "ntt_n16":
         unit, metric = "limb-NTTs/s", "forward+inverse negacyclic NTT throughput at N=2^16 (1 B200)"
         NPL = L + A
@@ -271,7 +273,17 @@ def run_ours(args):
         units_per_step = (wl.n_rot if wl.op == "hoisted" else B) * len(levels)
         rot_gs = [pow(5, 1 << r, 2 * N) for r in range(wl.n_rot)]  # steps 1, 2, 4, ...
 
+        if not args.no_graph and wl.op == "keyswitch" and B == 1 and len(levels) == 1:
+            l = levels[0]
+            graphs = [ctx.keyswitch_capture(ct[0, 0, :l], ct[0, 1, :l], l, keys[0], out[0, 0, :l], out[0, 1, :l])
+                      for ct, keys in sets]
+
         def step(k):
+            # graph replay, except every PROF_EVERY-th step: a direct call that
+            # carries the per-kernel events (the sampled roofline timing)
+            if graphs is not None and k % PROF_EVERY:
+                graphs[k % nsets].launch(stream)
+                return
             ct, keys = sets[k % nsets]
             for l in levels:
                 lN = l * N
@@ -303,9 +315,9 @@ def run_ours(args):
     if dist:
         dist.barrier()
     prof = args.workload != "ntt_n16"
-    PROF_EVERY = 10  # sampled steps carry per-kernel events; the rest run uninstrumented
     if prof:
-        ctx.profile_begin(args.steps * len(levels), PROF_EVERY)
+        # with graphs every direct call is a sampled one
+        ctx.profile_begin(args.steps * len(levels), 1 if graphs is not None else PROF_EVERY)
     clocks = ClockSampler(local)
     clocks.start()
     torch.cuda.synchronize()
@@ -333,7 +345,9 @@ def run_ours(args):
                       f"{wl.n_ct} ct/step, levels {levels[0]}..{levels[-1]}, key a-half "
                       f"{'regenerated in-kernel (ChaCha12)' if regen else 'stored in HBM'}",
                       "l2": f"inputs rotated over {nsets} sets of {per_set / 1e6:.1f} MB (> 126 MB L2)",
-                      "parallelism": f"replicas x{world}"},
+                      "parallelism": f"replicas x{world}",
+                      "launch": "CUDA graph replay" if args.workload != "ntt_n16" and graphs is not None
+                      else "library calls"},
            "gpu_launches": launches_per_step * args.steps
            - (0 if (os.environ.get("PC_NO_OVERLAP") or not prof) else ncalls), "clocks": clk}
 
@@ -540,6 +554,8 @@ def main():
                     choices=["rot1_n16", "relin_n12", "batch16_n16", "ntt_n16", "sweep_n17", "rotate_n16",
                              "hoisted8_n16", "relin_mul_n12", "relin_mul_n16"])
     ap.add_argument("--keys", default="regen", choices=["regen", "stored"])
+    ap.add_argument("--no-graph", action="store_true",
+                    help="call pc_keyswitch every step instead of replaying a CUDA graph of it")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")

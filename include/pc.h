@@ -171,6 +171,23 @@ int pc_keyswitch(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l
 int pc_keyswitch_batch(pc_ctx *ctx, const uint32_t *ct, uint32_t B, uint32_t l,
                        const pc_ksk *keys, uint32_t *out, pc_stream stream);
 
+/* CUDA graph of one pc_keyswitch: pc_keyswitch_capture records the launches
+ * of a key switch with these exact buffers, key and the context's current
+ * workspace (including the internal stream's ModDown branch) into an
+ * executable graph; pc_graph_launch replays it on `stream` (asynchronous),
+ * computing exactly what pc_keyswitch computes, with one host call instead of
+ * six launches and the fork/join events.  The buffers, the key's device
+ * halves and the workspace must stay valid and unchanged in place while the
+ * graph is used; calls sharing the context and workspace must still be
+ * ordered on one stream.  Same arguments and status codes as pc_keyswitch
+ * (out: the new graph, NULL on error).  The pages have no counterpart of
+ * these calls. */
+typedef struct pc_graph pc_graph;
+int pc_keyswitch_capture(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
+                         uint32_t *c0o, uint32_t *c1o, pc_graph **out);
+int pc_graph_launch(pc_graph *graph, pc_stream stream);
+void pc_graph_destroy(pc_graph *graph);
+
 /* Key switches of n ciphertexts held in HOST memory: ct and out are host
  * arrays [n][2][l][N] (c0 then c1 of each ciphertext, natural layout as in
  * device calls); keys: host array of n keys (device 'b' halves, as in

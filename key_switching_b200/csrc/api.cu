@@ -657,11 +657,12 @@ static cudaError_t ks_finish(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz,
 // shared body of the key-switching calls: B ciphertexts whose c0 / c1 /
 // outputs sit at stride `cz` words.
 static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u32 l, const pc_ksk *keys,
-                          u32 B, u32 *o0, u32 *o1, cudaStream_t s, const KsInput &in = KsInput{}) {
+                          u32 B, u32 *o0, u32 *o1, cudaStream_t s, const KsInput &in = KsInput{},
+                          bool profile = true) {
     const bool regen = keys[0].a == nullptr;
     for (u32 b = 1; b < B; ++b)
         if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
-    cudaEvent_t *ev = profile_slot(c);
+    cudaEvent_t *ev = profile ? profile_slot(c) : nullptr;
     cudaError_t e = ks_modup(c, c1, cz, l, B, B, in, s, ev);
     if (e == cudaSuccess) e = ks_finish(c, c0, c1, cz, l, keys, B, B, o0, o1, cz, in, s, ev);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
@@ -681,6 +682,70 @@ int pc_keyswitch(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, 
     if (int r = need_ws(c, l, 1)) return r;
     DeviceGuard dg(c->device);
     return keyswitch_core(c, c0, c1, 0, l, k, 1, c0o, c1o, (cudaStream_t)stream);
+}
+
+// An executable graph of one key switch (fixed buffers, workspace and key).
+struct pc_graph {
+    pc_ctx *ctx;
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+};
+
+int pc_keyswitch_capture(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
+                         uint32_t *c0o, uint32_t *c1o, pc_graph **out) {
+    if (!out) return PC_E_ARG;
+    *out = nullptr;
+    if (!c || !c0 || !c1 || !c0o || !c1o || l < 1 || l > c->L) return PC_E_ARG;
+    if (int r = check_ksk(c, k)) return r;
+    if (!aligned16(c0) || !aligned16(c1) || !aligned16(c0o) || !aligned16(c1o)) return PC_E_ALIGN;
+    if (int r = need_ws(c, l, 1)) return r;
+    DeviceGuard dg(c->device);
+    cudaStream_t cs = nullptr;
+    cudaError_t e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) {
+        cudaStreamDestroy(cs);
+        return cuda_fail(e);
+    }
+    // the same launches as pc_keyswitch (the internal stream's branch is
+    // forked from and joined back into the capturing stream), no profiling
+    int rc = keyswitch_core(c, c0, c1, 0, l, k, 1, c0o, c1o, cs, KsInput{}, false);
+    cudaGraph_t g = nullptr;
+    e = cudaStreamEndCapture(cs, &g);
+    cudaStreamDestroy(cs);
+    if (rc == PC_OK && e != cudaSuccess) rc = cuda_fail(e);
+    cudaGraphExec_t x = nullptr;
+    if (rc == PC_OK) {
+        e = cudaGraphInstantiate(&x, g, 0);
+        if (e != cudaSuccess) rc = cuda_fail(e);
+    }
+    if (rc != PC_OK) {
+        if (g) cudaGraphDestroy(g);
+        return rc;
+    }
+    *out = new (std::nothrow) pc_graph{c, g, x};
+    if (!*out) {
+        cudaGraphExecDestroy(x);
+        cudaGraphDestroy(g);
+        return PC_E_ARG;
+    }
+    return PC_OK;
+}
+
+int pc_graph_launch(pc_graph *gr, pc_stream stream) {
+    if (!gr) return PC_E_ARG;
+    DeviceGuard dg(gr->ctx->device);
+    const cudaError_t e = cudaGraphLaunch(gr->exec, (cudaStream_t)stream);
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
+void pc_graph_destroy(pc_graph *gr) {
+    if (!gr) return;
+    DeviceGuard dg(gr->ctx->device);
+    cudaGraphExecDestroy(gr->exec);
+    cudaGraphDestroy(gr->graph);
+    delete gr;
 }
 
 int pc_keyswitch_batch(pc_ctx *c, const uint32_t *ct, uint32_t B, uint32_t l, const pc_ksk *keys,

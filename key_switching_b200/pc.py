@@ -23,7 +23,8 @@ EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_wor
            "pc_set_workspace", "pc_ntt_fwd", "pc_ntt_inv", "pc_modup", "pc_keyswitch_inner",
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
            "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc",
-           "pc_rotate", "pc_rotate_hoisted", "pc_relinearize", "pc_keyswitch_host", "pc_host_workspace_bytes")
+           "pc_rotate", "pc_rotate_hoisted", "pc_relinearize", "pc_keyswitch_host", "pc_host_workspace_bytes",
+           "pc_keyswitch_capture", "pc_graph_launch", "pc_graph_destroy")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
@@ -90,6 +91,12 @@ def lib():
         L.pc_keyswitch_host.restype = i32
         L.pc_host_workspace_bytes.argtypes = [vp, u32]
         L.pc_host_workspace_bytes.restype = sz
+        L.pc_keyswitch_capture.argtypes = [vp, vp, vp, u32, ctypes.POINTER(_Ksk), vp, vp, ctypes.POINTER(vp)]
+        L.pc_keyswitch_capture.restype = i32
+        L.pc_graph_launch.argtypes = [vp, vp]
+        L.pc_graph_launch.restype = i32
+        L.pc_graph_destroy.argtypes = [vp]
+        L.pc_graph_destroy.restype = None
         L.pc_expand_a.argtypes = [vp, ctypes.c_char_p, u32, vp, vp]
         L.pc_expand_a.restype = i32
         L.pc_check.argtypes = [vp]
@@ -161,6 +168,29 @@ def microbench(kind: int, iters: int = 4096, device: int = 0) -> float:
     out = ctypes.c_double()
     _ok(lib().pc_microbench(device, kind, iters, ctypes.byref(out)), "pc_microbench")
     return out.value
+
+
+class Graph:
+    """An executable CUDA graph of one key switch (pc_keyswitch_capture); keeps
+    the captured buffers alive."""
+
+    def __init__(self, handle, keep):
+        self._h = handle
+        self._keep = keep
+
+    def launch(self, stream=None):
+        _ok(lib().pc_graph_launch(self._h, _stream(stream)), "pc_graph_launch")
+
+    def close(self):
+        if self._h:
+            lib().pc_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class KSK:
@@ -296,6 +326,14 @@ class Context:
         arr = (_Ksk * n)(*[k._c() for k in keys])
         _ok(lib().pc_keyswitch_host(self._h, _hptr(ct), n, l, arr, _hptr(out), _stream(stream)),
             "pc_keyswitch_host")
+
+    def keyswitch_capture(self, c0, c1, l: int, key: KSK, c0o, c1o) -> "Graph":
+        """A CUDA graph of pc_keyswitch on these buffers (replay with Graph.launch)."""
+        k = key._c()
+        h = ctypes.c_void_p()
+        _ok(lib().pc_keyswitch_capture(self._h, _ptr(c0), _ptr(c1), l, ctypes.byref(k), _ptr(c0o), _ptr(c1o),
+                                       ctypes.byref(h)), "pc_keyswitch_capture")
+        return Graph(h, (c0, c1, key, c0o, c1o))
 
     def relinearize(self, x, y, l: int, key: KSK, out, stream=None):
         k = key._c()
