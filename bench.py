@@ -273,9 +273,24 @@ def run_ours(args):
         units_per_step = (wl.n_rot if wl.op == "hoisted" else B) * len(levels)
         rot_gs = [pow(5, 1 << r, 2 * N) for r in range(wl.n_rot)]  # steps 1, 2, 4, ...
 
-        if not args.no_graph and wl.op == "keyswitch" and B == 1 and len(levels) == 1:
-            l = levels[0]
-            graphs = [ctx.keyswitch_capture(ct[0, 0, :l], ct[0, 1, :l], l, keys[0], out[0, 0, :l], out[0, 1, :l])
+        def run_op(ct, keys, st):
+            """One step's library calls on stream st."""
+            for l in levels:
+                if wl.op == "rotate":
+                    ctx.rotate(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs[0], keys[0], out[0, 0, :l], out[0, 1, :l], st)
+                elif wl.op == "hoisted":
+                    ctx.rotate_hoisted(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs, keys, out[:, :, :l], st)
+                elif wl.op == "relin":
+                    ctx.relinearize(ct[0, :, :l], ct[1, :, :l], l, keys[0], out[0, :, :l], st)
+                elif B == 1:
+                    # level-l ciphertext = the first l limbs of each half
+                    ctx.keyswitch(ct[0, 0, :l], ct[0, 1, :l], l, keys[0], out[0, 0, :l], out[0, 1, :l], st)
+                else:
+                    ctx.keyswitch_batch(ct, B, l, keys, out, st)
+
+        # one CUDA graph of a step per input set (single-ciphertext workloads)
+        if not args.no_graph and B == 1 and len(levels) == 1:
+            graphs = [ctx.capture(lambda st, ct=ct, keys=keys: run_op(ct, keys, st), keep=(ct, keys))
                       for ct, keys in sets]
 
         def step(k):
@@ -285,22 +300,7 @@ def run_ours(args):
                 graphs[k % nsets].launch(stream)
                 return
             ct, keys = sets[k % nsets]
-            for l in levels:
-                lN = l * N
-                if wl.op == "rotate":
-                    ctx.rotate(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs[0], keys[0], out[0, 0, :l], out[0, 1, :l],
-                               stream)
-                elif wl.op == "hoisted":
-                    ctx.rotate_hoisted(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs, keys, out[:, :, :l], stream)
-                elif wl.op == "relin":
-                    ctx.relinearize(ct[0, :, :l], ct[1, :, :l], l, keys[0], out[0, :, :l], stream)
-                elif B == 1:
-                    # level-l ciphertext = the first l limbs of each half
-                    c0 = ct[0, 0, :l]
-                    c1 = ct[0, 1, :l]
-                    ctx.keyswitch(c0, c1, l, keys[0], out[0, 0, :l], out[0, 1, :l], stream)
-                else:
-                    ctx.keyswitch_batch(ct, B, l, keys, out, stream)
+            run_op(ct, keys, stream)
         # 6 launches per key switch (the inner product splits in two when the
         # ModDown branch overlaps), 5 in the instrumented (serial) calls
         launches_per_step = (5 if os.environ.get("PC_NO_OVERLAP") else 6) * len(levels)

@@ -185,6 +185,17 @@ int pc_keyswitch_batch(pc_ctx *ctx, const uint32_t *ct, uint32_t B, uint32_t l,
 typedef struct pc_graph pc_graph;
 int pc_keyswitch_capture(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
                          uint32_t *c0o, uint32_t *c1o, pc_graph **out);
+
+/* General capture: pc_capture_begin returns, in *capture_stream, a stream in
+ * capture mode; the device-buffer calls (pc_keyswitch, pc_rotate,
+ * pc_rotate_hoisted, pc_relinearize, pc_keyswitch_batch, the NTTs, ...) made
+ * on it by this host thread are recorded, not run; pc_capture_end turns them
+ * into an executable graph (*out; pass NULL to abandon the capture).  One
+ * capture per context at a time (else PC_E_ARG).  Per-kernel profiling
+ * events are not recorded in captured calls.  The same rules as for
+ * pc_keyswitch_capture hold for the graph's buffers. */
+int pc_capture_begin(pc_ctx *ctx, pc_stream *capture_stream);
+int pc_capture_end(pc_ctx *ctx, pc_graph **out);
 int pc_graph_launch(pc_graph *graph, pc_stream stream);
 void pc_graph_destroy(pc_graph *graph);
 

@@ -432,6 +432,11 @@ void pc_ctx_destroy(pc_ctx *c) {
     for (cudaEvent_t ev : {c->ev_start, c->ev_in[0], c->ev_in[1], c->ev_done[0], c->ev_done[1], c->ev_out[0],
                            c->ev_out[1]})
         if (ev) cudaEventDestroy(ev);
+    if (c->cap) {  // a capture left open
+        cudaGraph_t g = nullptr;
+        if (cudaStreamEndCapture(c->cap, &g) == cudaSuccess && g) cudaGraphDestroy(g);
+        cudaStreamDestroy(c->cap);
+    }
     if (c->dev_block) cudaFree(c->dev_block);
     delete c;
 }
@@ -662,7 +667,9 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
     const bool regen = keys[0].a == nullptr;
     for (u32 b = 1; b < B; ++b)
         if ((keys[b].a == nullptr) != regen) return PC_E_ARG;
-    cudaEvent_t *ev = profile ? profile_slot(c) : nullptr;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (profile && cudaStreamIsCapturing(s, &cap) != cudaSuccess) cap = cudaStreamCaptureStatusNone;
+    cudaEvent_t *ev = profile && cap == cudaStreamCaptureStatusNone ? profile_slot(c) : nullptr;
     cudaError_t e = ks_modup(c, c1, cz, l, B, B, in, s, ev);
     if (e == cudaSuccess) e = ks_finish(c, c0, c1, cz, l, keys, B, B, o0, o1, cz, in, s, ev);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
@@ -691,38 +698,42 @@ struct pc_graph {
     cudaGraphExec_t exec;
 };
 
-int pc_keyswitch_capture(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
-                         uint32_t *c0o, uint32_t *c1o, pc_graph **out) {
-    if (!out) return PC_E_ARG;
-    *out = nullptr;
-    if (!c || !c0 || !c1 || !c0o || !c1o || l < 1 || l > c->L) return PC_E_ARG;
-    if (int r = check_ksk(c, k)) return r;
-    if (!aligned16(c0) || !aligned16(c1) || !aligned16(c0o) || !aligned16(c1o)) return PC_E_ALIGN;
-    if (int r = need_ws(c, l, 1)) return r;
+int pc_capture_begin(pc_ctx *c, pc_stream *capture_stream) {
+    if (!c || !capture_stream || c->cap) return PC_E_ARG;
     DeviceGuard dg(c->device);
     cudaStream_t cs = nullptr;
     cudaError_t e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
-    if (e != cudaSuccess) return cuda_fail(e);
-    e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+    if (e == cudaSuccess) e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) {
-        cudaStreamDestroy(cs);
+        if (cs) cudaStreamDestroy(cs);
         return cuda_fail(e);
     }
-    // the same launches as pc_keyswitch (the internal stream's branch is
-    // forked from and joined back into the capturing stream), no profiling
-    int rc = keyswitch_core(c, c0, c1, 0, l, k, 1, c0o, c1o, cs, KsInput{}, false);
+    c->cap = cs;
+    *capture_stream = (pc_stream)cs;
+    return PC_OK;
+}
+
+int pc_capture_end(pc_ctx *c, pc_graph **out) {
+    if (out) *out = nullptr;
+    if (!c || !c->cap) return PC_E_ARG;
+    DeviceGuard dg(c->device);
     cudaGraph_t g = nullptr;
-    e = cudaStreamEndCapture(cs, &g);
-    cudaStreamDestroy(cs);
-    if (rc == PC_OK && e != cudaSuccess) rc = cuda_fail(e);
-    cudaGraphExec_t x = nullptr;
-    if (rc == PC_OK) {
-        e = cudaGraphInstantiate(&x, g, 0);
-        if (e != cudaSuccess) rc = cuda_fail(e);
-    }
-    if (rc != PC_OK) {
+    cudaError_t e = cudaStreamEndCapture(c->cap, &g);
+    cudaStreamDestroy(c->cap);
+    c->cap = nullptr;
+    if (e != cudaSuccess) {
         if (g) cudaGraphDestroy(g);
-        return rc;
+        return cuda_fail(e);
+    }
+    if (!out) {  // capture abandoned
+        cudaGraphDestroy(g);
+        return PC_OK;
+    }
+    cudaGraphExec_t x = nullptr;
+    e = cudaGraphInstantiate(&x, g, 0);
+    if (e != cudaSuccess) {
+        cudaGraphDestroy(g);
+        return cuda_fail(e);
     }
     *out = new (std::nothrow) pc_graph{c, g, x};
     if (!*out) {
@@ -731,6 +742,24 @@ int pc_keyswitch_capture(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint
         return PC_E_ARG;
     }
     return PC_OK;
+}
+
+int pc_keyswitch_capture(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, const pc_ksk *k,
+                         uint32_t *c0o, uint32_t *c1o, pc_graph **out) {
+    if (!out) return PC_E_ARG;
+    *out = nullptr;
+    if (!c || !c0 || !c1 || !c0o || !c1o || l < 1 || l > c->L) return PC_E_ARG;
+    if (int r = check_ksk(c, k)) return r;
+    if (!aligned16(c0) || !aligned16(c1) || !aligned16(c0o) || !aligned16(c1o)) return PC_E_ALIGN;
+    if (int r = need_ws(c, l, 1)) return r;
+    pc_stream cs = nullptr;
+    if (int r = pc_capture_begin(c, &cs)) return r;
+    const int rc = pc_keyswitch(c, c0, c1, l, k, c0o, c1o, cs);
+    if (rc != PC_OK) {
+        pc_capture_end(c, nullptr);
+        return rc;
+    }
+    return pc_capture_end(c, out);
 }
 
 int pc_graph_launch(pc_graph *gr, pc_stream stream) {

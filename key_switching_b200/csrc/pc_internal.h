@@ -84,6 +84,8 @@ struct pc_ctx {
     // slot, "input landed", "key switch done" and "output copied" events
     cudaStream_t h2d, d2h;
     cudaEvent_t ev_start, ev_in[2], ev_done[2], ev_out[2];
+    // stream in capture mode between pc_capture_begin and pc_capture_end
+    cudaStream_t cap;
     // per-kernel timing (pc_profile_begin / pc_profile_end)
     cudaEvent_t *prof_ev;   // [prof_max][PC_PROFILE_STAGES + 1]
     uint32_t prof_max, prof_used, prof_every, prof_seen;

@@ -24,7 +24,7 @@ EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_wor
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
            "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc",
            "pc_rotate", "pc_rotate_hoisted", "pc_relinearize", "pc_keyswitch_host", "pc_host_workspace_bytes",
-           "pc_keyswitch_capture", "pc_graph_launch", "pc_graph_destroy")
+           "pc_keyswitch_capture", "pc_graph_launch", "pc_graph_destroy", "pc_capture_begin", "pc_capture_end")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
@@ -97,6 +97,10 @@ def lib():
         L.pc_graph_launch.restype = i32
         L.pc_graph_destroy.argtypes = [vp]
         L.pc_graph_destroy.restype = None
+        L.pc_capture_begin.argtypes = [vp, ctypes.POINTER(vp)]
+        L.pc_capture_begin.restype = i32
+        L.pc_capture_end.argtypes = [vp, ctypes.POINTER(vp)]
+        L.pc_capture_end.restype = i32
         L.pc_expand_a.argtypes = [vp, ctypes.c_char_p, u32, vp, vp]
         L.pc_expand_a.restype = i32
         L.pc_check.argtypes = [vp]
@@ -334,6 +338,19 @@ class Context:
         _ok(lib().pc_keyswitch_capture(self._h, _ptr(c0), _ptr(c1), l, ctypes.byref(k), _ptr(c0o), _ptr(c1o),
                                        ctypes.byref(h)), "pc_keyswitch_capture")
         return Graph(h, (c0, c1, key, c0o, c1o))
+
+    def capture(self, fn, keep=()) -> "Graph":
+        """Record the library calls fn(stream) makes on a capturing stream into a Graph."""
+        cs = ctypes.c_void_p()
+        _ok(lib().pc_capture_begin(self._h, ctypes.byref(cs)), "pc_capture_begin")
+        try:
+            fn(cs.value)
+        except BaseException:
+            lib().pc_capture_end(self._h, None)
+            raise
+        h = ctypes.c_void_p()
+        _ok(lib().pc_capture_end(self._h, ctypes.byref(h)), "pc_capture_end")
+        return Graph(h, keep)
 
     def relinearize(self, x, y, l: int, key: KSK, out, stream=None):
         k = key._c()

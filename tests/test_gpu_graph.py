@@ -76,3 +76,42 @@ def test_capture_errors(built, oracle):
         C.keyswitch_capture(c, c, 5, key, c, c)
     assert ei.value.code == -1
     C.check()
+
+
+def test_general_capture_of_several_calls(built, oracle):
+    """One graph holding a rotation, two hoisted rotations and a
+    relinearisation (pc_capture_begin / pc_capture_end), replayed twice:
+    bit-exact with the oracle."""
+    import torch
+    from key_switching_b200 import pc
+    P, C = G.contexts(oracle, 12, 4, 2, 30)
+    l = 4
+    C.ensure_workspace(l, 2)
+    seed, b = G.random_key(P, 23)
+    key = pc.KSK(seed, G.dev(b))
+    c0 = synth.uniform_residues(P.q, P.N, 96, 0)
+    c1 = synth.uniform_residues(P.q, P.N, 96, 1)
+    y = np.stack([synth.uniform_residues(P.q, P.N, 97, h) for h in range(2)])
+    d0, d1, dy, dx = G.dev(c0), G.dev(c1), G.dev(y), G.dev(np.stack([c0, c1]))
+    g = oracle.galois_elt(1, 12)
+    gs = [g, oracle.galois_elt(4, 12)]
+    r0, r1 = G.filled(l, P.N), G.filled(l, P.N)
+    hout = G.filled(2, 2, l, P.N)
+    rel = G.filled(2, l, P.N)
+
+    def calls(st):
+        C.rotate(d0, d1, l, g, key, r0, r1, st)
+        C.rotate_hoisted(d0, d1, l, gs, [key, key], hout, st)
+        C.relinearize(dx, dy, l, key, rel, st)
+    graph = C.capture(calls, keep=(d0, d1, dx, dy, key))
+    for _ in range(2):
+        graph.launch()
+        torch.cuda.synchronize()
+        w0, w1 = oracle.rotate(P, c0, c1, l, g, seed, b)
+        assert np.array_equal(G.host(r0), w0) and np.array_equal(G.host(r1), w1)
+        for i, (h0, h1) in enumerate(oracle.rotate_hoisted(P, c0, c1, l, gs, [seed, seed], [b, b])):
+            assert np.array_equal(G.host(hout[i, 0]), h0) and np.array_equal(G.host(hout[i, 1]), h1), i
+        w0, w1 = oracle.relinearize(P, c0, c1, y[0], y[1], l, seed, b)
+        assert np.array_equal(G.host(rel[0]), w0) and np.array_equal(G.host(rel[1]), w1)
+    graph.close()
+    C.check()
