@@ -346,8 +346,8 @@ def run_ours(args):
                       f"{'regenerated in-kernel (ChaCha12)' if regen else 'stored in HBM'}",
                       "l2": f"inputs rotated over {nsets} sets of {per_set / 1e6:.1f} MB (> 126 MB L2)",
                       "parallelism": f"replicas x{world}",
-                      "launch": "CUDA graph replay" if args.workload != "ntt_n16" and graphs is not None
-                      else "library calls"},
+                      "launch": f"CUDA graph replay (every {PROF_EVERY}th step a direct, instrumented call)"
+                      if graphs is not None else "library calls"},
            "gpu_launches": launches_per_step * args.steps
            - (0 if (os.environ.get("PC_NO_OVERLAP") or not prof) else ncalls), "clocks": clk}
 
