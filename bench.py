@@ -288,8 +288,9 @@ def run_ours(args):
                 else:
                     ctx.keyswitch_batch(ct, B, l, keys, out, st)
 
-        # one CUDA graph of a step per input set (single-ciphertext workloads)
-        if not args.no_graph and B == 1 and len(levels) == 1:
+        # one CUDA graph of a step per input set (single-ciphertext workloads;
+        # a level sweep is one graph of all its key switches)
+        if not args.no_graph and B == 1:
             graphs = [ctx.capture(lambda st, ct=ct, keys=keys: run_op(ct, keys, st), keep=(ct, keys))
                       for ct, keys in sets]
 
