@@ -255,6 +255,16 @@ def test_rotation_error_paths(built, oracle):
         C.rotate_hoisted(c0, c1, 4, [5, 25], [key, key], out)
     assert ei.value.code == -7
     C.ensure_workspace(4, 2)
+    with pytest.raises(pc.PCError) as ei:  # no rotation at all
+        C.rotate_hoisted(c0, c1, 4, [], [], out)
+    assert ei.value.code == -1
+    with pytest.raises(pc.PCError) as ei:  # no ciphertext at all
+        C.keyswitch_batch(out, 0, 4, [], out)
+    assert ei.value.code == -1
+    with pytest.raises(pc.PCError) as ei:
+        C.keyswitch_host(np.zeros((1, 2, 4, P.N), dtype=np.uint32), 0, 4, [],
+                         np.zeros((1, 2, 4, P.N), dtype=np.uint32))
+    assert ei.value.code == -1
     x = G.empty(2, 4, P.N)
     with pytest.raises(pc.PCError) as ei:
         C.relinearize(x, x, 4, key, x)
