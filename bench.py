@@ -1,20 +1,30 @@
 #!/usr/bin/env python
 """bench.py -- key-switches/s of CKKS hybrid key switching on B200.
 
-Default workload (one step = one key switch through pc_keyswitch):
+Default workload (one step = one key switch, pc_keyswitch):
   N=2^16, L=24 ciphertext primes + alpha=4 special primes (31-bit), dnum=6,
   one ciphertext at the top level (l=24), rotation key whose uniform half is
   regenerated in-kernel from its ChaCha12 seed; inputs are seeded uniform
   residues, rotated over enough (ciphertext, key) sets that the step's inputs
-  exceed the 126 MB L2.
+  exceed the 126 MB L2.  Each step replays a CUDA graph of the call captured
+  for its input set, except every 10th step, a direct call carrying per-kernel
+  CUDA events (the live roofline); --no-graph calls the library every step.
+
+Other workloads (--workload): relin_n12 (N=2^12 s^2 -> s key switch),
+batch16_n16 (16 ciphertexts, 16 keys, one batched call), ntt_n16 (64 x 28-limb
+forward + inverse NTTs), sweep_n17 (N=2^17, levels 40..1), rotate_n16 (one
+rotation), hoisted8_n16 (8 rotations sharing one ModUp), relin_mul_n12 /
+relin_mul_n16 (ciphertext product: tensor + relinearisation).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--keys regen|stored] [--impl ours|reference]
+                  [--keys regen|stored] [--no-graph] [--impl ours|reference]
 
-Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
-independent key switches (weak scaling, no data-path collective); the time is
-the max over ranks.  --impl reference times the plain CPU oracle on the host
-cores instead (rank 0 only).
+Prints one JSON line (rank 0) with the roofline of the dominant kernel, the
+oracle's single-core CPU baseline (single-GPU runs) and the end-to-end rate of
+host-resident ciphertexts through pc_keyswitch_host.  Multi-GPU (torchrun):
+every rank runs its own independent key switches (weak scaling, no data-path
+collective); the time is the max over ranks.  --impl reference times the plain
+CPU oracle on the host cores instead (rank 0 only).
 """
 from __future__ import annotations
 
