@@ -7,7 +7,7 @@ Default workload (one step = one key switch, pc_keyswitch):
   regenerated in-kernel from its ChaCha12 seed; inputs are seeded uniform
   residues, rotated over enough (ciphertext, key) sets that the step's inputs
   exceed the 126 MB L2.  Each step replays a CUDA graph of the call captured
-  for its input set, except every 10th step, a direct call carrying per-kernel
+  for its input set, except every 30th step, a direct call carrying per-kernel
   CUDA events (the live roofline); --no-graph calls the library every step.
 
 Other workloads (--workload): relin_n12 (N=2^12 s^2 -> s key switch),
@@ -238,7 +238,7 @@ def run_ours(args):
 
     launches_per_step = 5
     graphs = None
-    PROF_EVERY = 10  # sampled steps carry per-kernel events; the rest run uninstrumented
+    PROF_EVERY = 30  # sampled steps carry per-kernel events; the rest run uninstrumented
     if args.workload == "ntt_n16":
         unit, metric = "limb-NTTs/s", "forward+inverse negacyclic NTT throughput at N=2^16 (1 B200)"
         NPL = L + A
