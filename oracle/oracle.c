@@ -570,6 +570,78 @@ int or_relinearize(const or_params *P, const uint32_t *x0, const uint32_t *x1, c
 }
 
 /* ------------------------------------------------------------------ */
+/* baby-step giant-step linear transform                               */
+/* ------------------------------------------------------------------ */
+/* The homomorphic linear transform of CKKS bootstrapping's
+ * CoeffsToSlots / SlotsToCoeffs steps by the diagonal method with baby steps
+ * and giant steps (Halevi-Shoup diagonals; baby-step giant-step split as in
+ * Han-Ki 2020 and Chen-Chillotti-Song 2019), with hoisted baby steps:
+ *   bs_0 = (c0, c1);  bs_j = hoisted rotation of (c0, c1) by gb[j-1], j < n1
+ *                           (one ModUp of c1 shared by every baby step)
+ *   W_i  = sum_{j<n1} diag[i][j] (.) bs_j      (slot-wise, both halves)
+ *   out  = W_0 + sum_{1<=i<n2} rotation of W_i by gg[i-1]
+ * diag: [n2][n1][l][N] NTT-domain plaintexts (the caller's pre-rotated
+ * diagonals); baby key j-1 (seed_b + 32 (j-1), b_b[j-1]) switches
+ * s(X^gb[j-1]) -> s, giant key i-1 switches s(X^gg[i-1]) -> s.  The 'a'
+ * halves are regenerated (rounds).  out0, out1: [l][N]. */
+int or_linear_transform(const or_params *P, const uint32_t *c0, const uint32_t *c1, uint32_t l,
+                        uint32_t n1, const uint32_t *gb, const uint8_t *seed_b, const uint32_t *const *b_b,
+                        uint32_t n2, const uint32_t *gg, const uint8_t *seed_g, const uint32_t *const *b_g,
+                        const uint32_t *diag, int rounds, uint32_t *out0, uint32_t *out1) {
+    if (check_params(P, l) || n1 < 1 || n2 < 1) return -1;
+    uint32_t N = 1u << P->logN, al = P->alpha, beta = (l + al - 1) / al, ll = l + al;
+    size_t lN = (size_t)l * N;
+    uint32_t *ext = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)beta * ll * N);
+    uint32_t *bs = (uint32_t *)malloc(sizeof(uint32_t) * 2 * lN * n1);
+    uint32_t *w = (uint32_t *)malloc(sizeof(uint32_t) * 2 * lN);
+    uint32_t *r = (uint32_t *)malloc(sizeof(uint32_t) * 2 * lN);
+    int rc = or_modup(P, c1, l, ext);
+    /* baby steps */
+    memcpy(bs, c0, sizeof(uint32_t) * lN);
+    memcpy(bs + lN, c1, sizeof(uint32_t) * lN);
+    for (uint32_t j = 1; j < n1 && !rc; j++)
+        rc = or_rotate_hoisted_one(P, c0, ext, l, gb[j - 1], seed_b + 32 * (size_t)(j - 1), b_b[j - 1], NULL,
+                                   rounds, bs + 2 * lN * j, bs + 2 * lN * j + lN);
+    /* giant steps */
+    for (uint32_t i = 0; i < n2 && !rc; i++) {
+        for (uint32_t t = 0; t < l; t++) {
+            uint32_t q = P->q[t];
+            for (uint32_t n = 0; n < N; n++) {
+                size_t o = (size_t)t * N + n;
+                uint32_t v0 = 0, v1 = 0;
+                for (uint32_t j = 0; j < n1; j++) {
+                    uint32_t d = diag[((size_t)i * n1 + j) * lN + o];
+                    v0 = addm(v0, mulm(d, bs[2 * lN * j + o], q), q);
+                    v1 = addm(v1, mulm(d, bs[2 * lN * j + lN + o], q), q);
+                }
+                w[o] = v0;
+                w[lN + o] = v1;
+            }
+        }
+        if (i == 0) {
+            memcpy(out0, w, sizeof(uint32_t) * lN);
+            memcpy(out1, w + lN, sizeof(uint32_t) * lN);
+            continue;
+        }
+        rc = or_rotate(P, w, w + lN, l, gg[i - 1], seed_g + 32 * (size_t)(i - 1), b_g[i - 1], NULL, rounds, r,
+                       r + lN);
+        for (uint32_t t = 0; t < l && !rc; t++) {
+            uint32_t q = P->q[t];
+            for (uint32_t n = 0; n < N; n++) {
+                size_t o = (size_t)t * N + n;
+                out0[o] = addm(out0[o], r[o], q);
+                out1[o] = addm(out1[o], r[lN + o], q);
+            }
+        }
+    }
+    free(r);
+    free(w);
+    free(bs);
+    free(ext);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
 /* key generation (the oracle side only; the library never generates)  */
 /* ------------------------------------------------------------------ */
 

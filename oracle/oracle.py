@@ -66,6 +66,8 @@ def lib():
         L.or_tensor.restype = i32
         L.or_relinearize.argtypes = [vp, vp, vp, vp, vp, u32, vp, vp, vp, i32, vp, vp]
         L.or_relinearize.restype = i32
+        L.or_linear_transform.argtypes = [vp, vp, vp, u32, u32, vp, vp, vp, u32, vp, vp, vp, vp, i32, vp, vp]
+        L.or_linear_transform.restype = i32
         L.or_negacyclic_mul.argtypes = [vp, vp, u32, vp]
         L.or_automorph.argtypes = [vp, u32, u32, vp]
         L.or_ksk_gen.argtypes = [vp, vp, vp, vp, vp, i32, vp]
@@ -312,6 +314,38 @@ def relinearize(P: Params, x0, x1, y0, y1, l: int, seed: bytes, b: np.ndarray, a
                             _p(c0o), _p(c1o)) != 0:
         raise ValueError("or_relinearize: bad arguments")
     return c0o, c1o
+
+
+def linear_transform(P: Params, c0: np.ndarray, c1: np.ndarray, l: int, diag: np.ndarray,
+                     gb, seeds_b, bs_b, gg, seeds_g, bs_g, rounds: int = ROUNDS):
+    """Baby-step giant-step linear transform with hoisted baby steps:
+    out = sum_i rot_{gg_i}( sum_j diag[i][j] (.) rot_{gb_j}(ct) ), with the
+    identity as baby step 0 and giant step 0.  diag: [n2][n1][l][N]; gb, seeds_b,
+    bs_b: the n1-1 baby rotations (Galois elements, ChaCha seeds, key 'b'
+    halves); gg, seeds_g, bs_g: the n2-1 giant rotations.  Returns (c0', c1')."""
+    diag = np.ascontiguousarray(diag, dtype=np.uint32)
+    n2, n1 = int(diag.shape[0]), int(diag.shape[1])
+    assert diag.shape == (n2, n1, l, P.N)
+    assert len(gb) == len(seeds_b) == len(bs_b) == n1 - 1 and len(gg) == len(seeds_g) == len(bs_g) == n2 - 1
+    c0 = np.ascontiguousarray(c0, dtype=np.uint32)
+    c1 = np.ascontiguousarray(c1, dtype=np.uint32)
+    keep = []
+
+    def keys(gs, seeds, bs):
+        ga = np.ascontiguousarray(np.asarray(gs, dtype=np.uint32).reshape(-1))
+        sa = np.frombuffer(b"".join(bytes(x) for x in seeds) or b"\0", dtype=np.uint8).copy()
+        arrs = [np.ascontiguousarray(b, dtype=np.uint32) for b in bs]
+        ptrs = (ctypes.c_void_p * max(1, len(arrs)))(*[a.ctypes.data for a in arrs])
+        keep.extend([ga, sa, arrs, ptrs])
+        return _p(ga), _p(sa), ptrs
+    gbp, sbp, bbp = keys(gb, seeds_b, bs_b)
+    ggp, sgp, bgp = keys(gg, seeds_g, bs_g)
+    o0 = np.zeros((l, P.N), dtype=np.uint32)
+    o1 = np.zeros((l, P.N), dtype=np.uint32)
+    if lib().or_linear_transform(P.ptr, _p(c0), _p(c1), l, n1, gbp, sbp, bbp, n2, ggp, sgp, bgp, _p(diag),
+                                 rounds, _p(o0), _p(o1)) != 0:
+        raise ValueError("or_linear_transform: bad arguments")
+    return o0, o1
 
 
 def negacyclic_mul(a: np.ndarray, b: np.ndarray, logN: int) -> np.ndarray:
