@@ -6,25 +6,30 @@ Default workload (one step = one key switch, pc_keyswitch):
   one ciphertext at the top level (l=24), rotation key whose uniform half is
   regenerated in-kernel from its ChaCha12 seed; inputs are seeded uniform
   residues, rotated over enough (ciphertext, key) sets that the step's inputs
-  exceed the 126 MB L2.  Each step replays a CUDA graph of the call captured
-  for its input set, except every 30th step, a direct call carrying per-kernel
-  CUDA events (the live roofline); --no-graph calls the library every step.
+  exceed the 126 MB L2.  Each timed step replays a CUDA graph of the call
+  captured for its input set (--no-graph calls the library every step).
+  After the timed region, a separate pass of at least 10 direct calls carries
+  per-kernel CUDA events; their medians give the dominant kernel's roofline.
 
 Other workloads (--workload): relin_n12 (N=2^12 s^2 -> s key switch),
-batch16_n16 (16 ciphertexts, 16 keys, one batched call), ntt_n16 (64 x 28-limb
-forward + inverse NTTs), sweep_n17 (N=2^17, levels 40..1), rotate_n16 (one
-rotation), hoisted8_n16 (8 rotations sharing one ModUp), relin_mul_n12 /
-relin_mul_n16 (ciphertext product: tensor + relinearisation).
+batch16_n16 (16 ciphertexts, 16 keys, one batched call; split across the
+ranks when run on several GPUs), ntt_n16 (64 x 28-limb forward + inverse
+NTTs), sweep_n17 (N=2^17, levels 40..1), rotate_n16 (one rotation),
+hoisted8_n16 (8 rotations sharing one ModUp), relin_mul_n12 / relin_mul_n16
+(ciphertext product: tensor + relinearisation).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--keys regen|stored] [--no-graph] [--impl ours|reference]
 
 Prints one JSON line (rank 0) with the roofline of the dominant kernel, the
-oracle's single-core CPU baseline (single-GPU runs) and the end-to-end rate of
-host-resident ciphertexts through pc_keyswitch_host.  Multi-GPU (torchrun):
-every rank runs its own independent key switches (weak scaling, no data-path
-collective); the time is the max over ranks.  --impl reference times the plain
-CPU oracle on the host cores instead (rank 0 only).
+oracle's CPU baseline on the host cores (single-GPU runs) and the end-to-end
+rate of host-resident ciphertexts through pc_keyswitch_host.  With --gpus N
+the script runs N ranks, one per GPU (started by torch.distributed.run, or by
+itself when launched as one process): every rank runs its own key switches
+(weak scaling, no data-path collective), except that the 16-pair batch is
+split across the ranks (strong scaling); the time is the max over ranks.
+--impl reference times the plain CPU oracle on the host cores instead (rank 0
+only).
 """
 from __future__ import annotations
 
@@ -42,10 +47,24 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 2**20
-# DRAM bytes (read + write) per launch of the roofline kernel, from one ncu
-# capture of the current kernel (profiles/k_inner_keyswitch_n16.md, cold
-# cache); None when the kernel has changed since the counters were taken.
-KERNEL_TRAFFIC = {("rot1_n16", "inner_chacha"): 104.93e6 + 5.13e6}
+# DRAM bytes (read + write) of one launch of the roofline kernel, recorded
+# from one ncu capture (--clock-control none, cold cache) of the kernel source
+# whose hash is given; reported only while the kernel sources still hash to
+# that value (otherwise the traffic is null: the counters are stale).
+KERNEL_TRAFFIC = {("rot1_n16", "inner_chacha"): (104.93e6 + 5.13e6, "0000000000000000")}
+KERNEL_SOURCES = ("kernels.cu", "ntt.cuh", "chacha.cuh", "modarith.cuh")
+
+
+def kernel_source_hash() -> str:
+    """First 16 hex digits of the SHA-256 of the kernel sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "key_switching_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 # A Shoup modular multiply is IMAD.HI + 2 IMAD on the 16-lane-per-partition
 # multiply-add pipe, and the high-half multiply occupies two issue slots:
 # 4 slots of 64 lanes/SM/clock (measured by pc_microbench kind 0 at 4.57 T/s)
@@ -204,6 +223,57 @@ def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: f
     return units_per_rank_step * steps * world / (max_ms * 1e-3)
 
 
+def shard(n_items: int, world: int, rank: int) -> range:
+    """The contiguous share of n_items independent units that rank `rank` of
+    `world` processes: sizes differ by at most one, every unit is in exactly
+    one share."""
+    lo = n_items * rank // world
+    hi = n_items * (rank + 1) // world
+    return range(lo, hi)
+
+
+def rank_plan(workload: str, n_ct: int, world: int, rank: int, local: int):
+    """What one rank runs: its device (the local rank's GPU) and the indices of
+    the workload's (ciphertext, key) pairs it key-switches.  A batch of
+    independent pairs is split across the ranks (strong scaling: the job's
+    total is fixed); every other workload runs whole on every rank (weak
+    scaling: replicas)."""
+    if workload == "batch16_n16":
+        return {"device": local, "items": shard(n_ct, world, rank), "scaling": "strong"}
+    return {"device": local, "items": range(n_ct), "scaling": "weak"}
+
+
+def launch_ranks(argv, n: int) -> int:
+    """Re-run this script as n ranks on this node (one process per GPU) when it
+    was started as a single process with --gpus n > 1; returns the launcher's
+    exit status.  Rank 0 prints the JSON line."""
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def workload_metric(wl) -> str:
+    """The metric line of a workload (the N=2^16 key switch carries the
+    headline metric's exact wording)."""
+    if wl.name == "ntt_n16":
+        return "forward+inverse negacyclic NTT throughput at N=2^16 (1 B200)"
+    if wl.name == "sweep_n17":
+        return "key-switches/s at N=2^17 level sweep 40..1 (1 B200)"
+    if wl.op in ("rotate", "hoisted"):
+        return (f"rotations/s at N=2^{wl.logN} ({'single' if wl.op == 'rotate' else f'{wl.n_rot} hoisted'}"
+                " rotation(s) per ciphertext; 1 B200)")
+    if wl.op == "relin":
+        return f"ciphertext products (tensor + relinearisation) per second at N=2^{wl.logN} (1 B200)"
+    if wl.logN == 16:
+        return "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline"
+    return f"key-switches/s at N=2^{wl.logN} (1 B200)"
+
+
 # --------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -214,6 +284,7 @@ def run_ours(args):
     from key_switching_b200 import pc, synth
 
     world, rank, local = dist_setup()
+    assert world == args.gpus, f"--gpus {args.gpus} but WORLD_SIZE={world}"
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -221,8 +292,9 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     wl = synth.WORKLOADS[args.workload]
+    plan = rank_plan(args.workload, wl.n_ct, world, rank, local)
     q, p = pc.chain(wl.logN, wl.bits, wl.L, wl.alpha)
-    ctx = pc.Context(wl.logN, q, p, device=local)
+    ctx = pc.Context(wl.logN, q, p, device=plan["device"])
     N, L, A = wl.N, wl.L, wl.alpha
     regen = args.keys == "regen"
     prim = q + p
@@ -236,11 +308,10 @@ def run_ours(args):
             a = dev(np.stack([synth.uniform_residues(prim, N, seed_id, 0xA, j) for j in range(wl.dnum)]))
         return pc.KSK(synth.chacha_seed(seed_id, rank), dev(b), a)
 
-    launches_per_step = 5
     graphs = None
-    PROF_EVERY = 30  # sampled steps carry per-kernel events; the rest run uninstrumented
+    items = list(plan["items"])
     if args.workload == "ntt_n16":
-        unit, metric = "limb-NTTs/s", "forward+inverse negacyclic NTT throughput at N=2^16 (1 B200)"
+        unit, metric = "limb-NTTs/s", workload_metric(wl)
         NPL = L + A
         per_set = wl.n_ct * NPL * N * 4
         nsets = max(2, math.ceil(2 * L2_BYTES / per_set))
@@ -254,19 +325,11 @@ def run_ours(args):
         launches_per_step = 4
         levels = [L]
         work = None
+        run_op = None
     else:
-        unit, metric = "key-switches/s", "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline"
-        if args.workload == "sweep_n17":
-            metric = "key-switches/s at N=2^17 level sweep 40..1 (1 B200)"
-        if wl.op in ("rotate", "hoisted"):
-            unit = "rotations/s"
-            metric = (f"rotations/s at N=2^{wl.logN} ({'single' if wl.op == 'rotate' else f'{wl.n_rot} hoisted'}"
-                      " rotation(s) per ciphertext; 1 B200)")
-        elif wl.op == "relin":
-            unit = "relinearisations/s"
-            metric = f"ciphertext products (tensor + relinearisation) per second at N=2^{wl.logN} (1 B200)"
+        unit, metric = _unit(wl), workload_metric(wl)
         levels = list(wl.levels) if wl.levels else [L]
-        B = wl.n_ct
+        B = len(items)  # this rank's ciphertexts per step
         nk = wl.n_rot if wl.op == "hoisted" else B  # keys per step
         ctx.ensure_workspace(max(levels), max(B, min(wl.n_rot, 16)) if wl.op == "hoisted" else B)
         per_set = (B * (2 * L * N * 4) * (2 if wl.op == "relin" else 1)
@@ -275,9 +338,10 @@ def run_ours(args):
         sets = []
         nct = B * (2 if wl.op == "relin" else 1)
         for s in range(nsets):
-            keys = [make_key(1000 * s + k + 1) for k in range(nk)]
+            key_ids = items if wl.op != "hoisted" else range(nk)
+            keys = [make_key(1000 * s + k + 1) for k in key_ids]
             ct = dev(np.stack([np.stack([synth.uniform_residues(q, N, 50 + s, rank, k, h) for h in range(2)])
-                               for k in range(nct)]))
+                               for k in (items if wl.op != "relin" else range(nct))]))
             sets.append((ct, keys))
         out = torch.empty((max(B, wl.n_rot), 2, L, N), dtype=torch.int32, device="cuda")
         units_per_step = (wl.n_rot if wl.op == "hoisted" else B) * len(levels)
@@ -305,32 +369,23 @@ def run_ours(args):
                       for ct, keys in sets]
 
         def step(k):
-            # graph replay, except every PROF_EVERY-th step: a direct call that
-            # carries the per-kernel events (the sampled roofline timing)
-            if graphs is not None and k % PROF_EVERY:
+            if graphs is not None:
                 graphs[k % nsets].launch(stream)
-                return
-            ct, keys = sets[k % nsets]
-            run_op(ct, keys, stream)
+            else:
+                run_op(*sets[k % nsets], stream)
         # 6 launches per key switch (the inner product splits in two when the
-        # ModDown branch overlaps), 5 in the instrumented (serial) calls
+        # ModDown branch overlaps), 5 when the stages run serially
         launches_per_step = (5 if os.environ.get("PC_NO_OVERLAP") else 6) * len(levels)
-        if wl.op == "hoisted":  # one ModUp (2), then per rotation 4 (3 when serial)
-            launches_per_step = (2 + (3 if os.environ.get("PC_NO_OVERLAP") else 4) * wl.n_rot) * len(levels)
+        if wl.op == "hoisted":  # one ModUp (2), then per batch of up to 16 rotations 4 (3 when serial)
+            launches_per_step = (2 + (3 if os.environ.get("PC_NO_OVERLAP") else 4) * -(-wl.n_rot // 16)) \
+                * len(levels)
         work = [op_counts(wl, l, regen) for l in levels]
 
+    clocks = ClockSampler(local)
+    clocks.start()
     # warm-up, then exactly K timed steps between barriers
     for k in range(args.warmup):
         step(k)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    prof = args.workload != "ntt_n16"
-    if prof:
-        # with graphs every direct call is a sampled one
-        ctx.profile_begin(args.steps * len(levels), 1 if graphs is not None else PROF_EVERY)
-    clocks = ClockSampler(local)
-    clocks.start()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -342,77 +397,103 @@ def run_ours(args):
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    stage_ms, ncalls = ctx.profile_end() if prof else ({}, 0)
     ms = max_over_ranks(ms, dist, "cuda")
     value = whole_job_rate(units_per_step, args.steps, world, ms)
+    if plan["scaling"] == "strong":
+        # the ranks split one job's units: the job's units over the slowest rank's time
+        value = wl.n_ct * len(levels) * args.steps / (ms * 1e-3)
+
+    # per-kernel events: a separate pass of direct, instrumented calls after
+    # the timed region (each runs its kernels serially on the stream, with an
+    # event between consecutive kernels)
+    stage_calls = []
+    if run_op is not None and wl.op != "hoisted":
+        n_prof = max(10, min(args.steps, 30)) if len(levels) == 1 else 10
+        for k in range(n_prof):
+            ctx.profile_begin(len(levels), 1)
+            run_op(*sets[k % nsets], stream)
+            ms_k, n_k = ctx.profile_end()
+            if n_k:
+                stage_calls.append(ms_k)
+    clk = clocks.stop()
 
     res = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic (seeded uniform residues, "
-           "uniform key 'b' halves; ChaCha12 seeds)",
+           "scaling": plan["scaling"], "vs_baseline": None, "dtype": "u32",
+           "data": "synthetic (seeded uniform residues, uniform key 'b' halves; ChaCha12 seeds)",
            "config": {"workload": f"{wl.name}: N=2^{wl.logN}, L={L}, alpha={A}, dnum={wl.dnum}, "
                       f"{wl.n_ct} ct/step, levels {levels[0]}..{levels[-1]}, key a-half "
                       f"{'regenerated in-kernel (ChaCha12)' if regen else 'stored in HBM'}",
                       "l2": f"inputs rotated over {nsets} sets of {per_set / 1e6:.1f} MB (> 126 MB L2)",
-                      "parallelism": f"replicas x{world}",
-                      "launch": f"CUDA graph replay (every {PROF_EVERY}th step a direct, instrumented call)"
-                      if graphs is not None else "library calls"},
-           "gpu_launches": launches_per_step * args.steps
-           - (0 if (os.environ.get("PC_NO_OVERLAP") or not prof) else ncalls), "clocks": clk}
+                      "parallelism": (f"{wl.n_ct} (ciphertext, key) pairs split over {world} rank(s)"
+                                      if plan["scaling"] == "strong" else f"replicas x{world}"),
+                      "launch": "CUDA graph replay of every step" if graphs is not None else "library calls"},
+           "gpu_launches": launches_per_step * args.steps, "clocks": clk}
 
     if work is not None:
+        nct = B  # this rank's ciphertexts per step
         mm = sum(w["modmuls"] for w in work)
         by = sum(w["bytes"] for w in work)
-        sec_per_step = ms * 1e-3 / args.steps / world * world  # per rank
-        sm_mhz = clk.get("sm_mhz") or 1965.0
+        sec_per_step = ms * 1e-3 / args.steps
         peak_derived = SMS * IMAD_PER_SM_CLK * 1965e6 / MODMUL_IMAD
         try:
             peak_meas = pc.microbench(0, 2048, local) if rank == 0 else None
         except Exception:
             peak_meas = None
-        hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"] \
-            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 6650.0
+        hbm_src = "MEASURED_PEAKS.json"
+        try:
+            hbm = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
+        except (OSError, KeyError, ValueError):
+            hbm, hbm_src = 6650.0, "fallback 6650 GB/s (MEASURED_PEAKS.json absent)"
         t_roof = max(by / (hbm * 1e9), mm / peak_derived)
-        res["step_roofline"] = {"modmuls_per_step": mm * wl.n_ct, "hbm_bytes_per_step": by * wl.n_ct,
-                                "achieved_gbs": by * wl.n_ct / sec_per_step / 1e9,
-                                "achieved_tmodmul_s": mm * wl.n_ct / sec_per_step / 1e12,
-                                "t_roofline_us": t_roof * wl.n_ct * 1e6, "t_step_us": sec_per_step * 1e6,
-                                "frac": t_roof * wl.n_ct / sec_per_step,
+        res["step_roofline"] = {"modmuls_per_step": mm * nct, "hbm_bytes_per_step": by * nct,
+                                "achieved_gbs": by * nct / sec_per_step / 1e9,
+                                "achieved_tmodmul_s": mm * nct / sec_per_step / 1e12,
+                                "t_roofline_us": t_roof * nct * 1e6, "t_step_us": sec_per_step * 1e6,
+                                "frac": t_roof * nct / sec_per_step,
                                 "modmul_peak_derived": peak_derived,
-                                "modmul_peak_microbench": peak_meas, "hbm_peak_gbs": hbm}
-        if stage_ms and ncalls:
+                                "modmul_peak_microbench": peak_meas, "hbm_peak_gbs": hbm, "hbm_peak_source": hbm_src}
+        peak_ops = SMS * ISSUE_LANES_PER_SM_CLK * 1965e6
+        if stage_calls:
             smm = {}
             for l in levels:
                 for kname, v in stage_modmuls(wl.logN, L, A, l).items():
-                    smm[kname] = smm.get(kname, 0) + v * wl.n_ct
+                    smm[kname] = smm.get(kname, 0) + v * nct
             # integer lane operations per stage: 4 per modular multiply, 592
             # per ChaCha12 block (the inner-product stage regenerates a)
-            blocks = sum(w["chacha_blocks"] for w in work) * wl.n_ct
+            blocks = sum(w["chacha_blocks"] for w in work) * nct
             sops = {k: MODMUL_IMAD * v for k, v in smm.items()}
             sops["inner_chacha"] += CHACHA_OPS * blocks
-            peak_ops = SMS * ISSUE_LANES_PER_SM_CLK * 1965e6
-            tot = sum(stage_ms.values())
-            top = max(stage_ms, key=stage_ms.get)
-            per_launch_s = stage_ms[top] * 1e-3 / ncalls * len(levels)
-            ach = sops[top] / per_launch_s
+            med = {k: statistics.median(c[k] for c in stage_calls) for k in stage_calls[0]}
+            tot = sum(med.values())
+            top = max(med, key=med.get)
+            per_launch_s = med[top] * 1e-3 / len(levels)
+            ach = sops[top] / len(levels) / per_launch_s
+            tr = KERNEL_TRAFFIC.get((args.workload, top)) if regen else None
+            src_hash = kernel_source_hash()
+            traffic = tr[0] if tr and tr[1] == src_hash else None
             res["roofline"] = {"bound": "alu", "kernel": top, "achieved": ach / 1e12,
                                "peak": peak_ops / 1e12, "unit": "Tintop/s",
                                "frac": ach / peak_ops,
-                               "traffic": KERNEL_TRAFFIC.get((args.workload, top)) if regen else None,
-                               "share": stage_ms[top] / tot if tot else None,
+                               "traffic": traffic,
+                               "traffic_source": (f"ncu capture of the kernel sources hashing to {tr[1]} "
+                                                  "(recorded constant, not measured in this run)"
+                                                  if traffic is not None else
+                                                  f"none recorded for kernel sources {src_hash}"),
+                               "share": med[top] / tot if tot else None,
                                "ops_per_launch": sops[top] / len(levels),
-                               "modmul_frac": smm[top] / per_launch_s / peak_derived,
+                               "modmul_frac": smm[top] / len(levels) / per_launch_s / peak_derived,
                                "peak_source": "derived: 148 SMs x 128 issued 32-bit lane ops/clk (4 partitions x "
                                               "32; ALU + multiply-add pipes) x 1965 MHz; ops = 4 per Shoup "
                                               "modular multiply + 592 per ChaCha12 block"}
-            res["stage_ms_per_step"] = {k: v / ncalls * len(levels) for k, v in stage_ms.items()}
-            res["stage_sampling"] = f"{ncalls} of {args.steps * len(levels)} calls instrumented (every {PROF_EVERY}th)"
+            res["stage_ms_per_step"] = med
+            res["stage_sum_ms"] = tot
+            res["stage_sampling"] = (f"median of {len(stage_calls)} direct instrumented steps run after the timed "
+                                     "region (stages serial, one event between consecutive kernels)")
         else:
             # no per-kernel events on this path (hoisted rotations): the whole step
-            peak_ops = SMS * ISSUE_LANES_PER_SM_CLK * 1965e6
-            ops = (MODMUL_IMAD * mm + CHACHA_OPS * sum(w["chacha_blocks"] for w in work)) * wl.n_ct
+            ops = (MODMUL_IMAD * mm + CHACHA_OPS * sum(w["chacha_blocks"] for w in work)) * nct
             ach = ops / sec_per_step
             res["roofline"] = {"bound": "alu", "kernel": "whole step", "achieved": ach / 1e12,
                                "peak": peak_ops / 1e12, "unit": "Tintop/s", "frac": ach / peak_ops,
@@ -446,111 +527,199 @@ def run_ours(args):
         res["e2e"] = {"value": whole_job_rate(1, ke, world, ems), "unit": unit,
                       "h2d_bytes_per_step": 2 * l * N * 4, "d2h_bytes_per_step": 2 * l * N * 4}
 
-    # the oracle's CPU baseline: rank 0 of a single-GPU run only
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in ("rot1_n16", "relin_n12"):
-        res["cpu_baseline"] = cpu_baseline(wl, q, p, budget_s=args.cpu_budget)
-
+    for g in graphs or []:
+        g.close()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+    # the oracle's CPU baseline: rank 0 of a single-GPU run only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in CPU_BASELINE_WORKLOADS:
+        res["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(res), flush=True)
 
 
 # ------------------------------------------------------------ oracle timing
+# Everything below runs the CPU oracle only; it builds its own basis with the
+# oracle's prime generator and imports nothing of the CUDA library.
 
-def _oracle_inputs(wl, q, p):
-    import numpy as np
-    from key_switching_b200 import synth
-    from oracle import oracle as O
-    P = O.Params(wl.logN, q, p)
-    prim = [P.prime(g) for g in range(P.L + P.alpha)]
-    b = np.stack([synth.uniform_residues(prim, P.N, 1, 0xB, j) for j in range(P.dnum)])
-    l = wl.L
-    c0 = synth.uniform_residues(P.q[:l], P.N, 50, 0, 0, 0)
-    c1 = synth.uniform_residues(P.q[:l], P.N, 50, 0, 0, 1)
-    return O, P, b, c0, c1, l, synth.chacha_seed(1, 0)
-
-
-def oracle_step(wl, O, P, b, c0, c1, l, seed):
-    """One unit batch of the workload's operation on the oracle; returns the
-    number of operations done (n_rot for hoisted rotations, else 1)."""
-    from key_switching_b200 import synth
-    if wl.op == "rotate":
-        O.rotate(P, c0, c1, l, pow(5, 1, 2 * P.N), seed, b)
-    elif wl.op == "hoisted":
-        gs = [pow(5, 1 << r, 2 * P.N) for r in range(wl.n_rot)]
-        O.rotate_hoisted(P, c0, c1, l, gs, [seed] * wl.n_rot, [b] * wl.n_rot)
-        return wl.n_rot
-    elif wl.op == "relin":
-        y0 = synth.uniform_residues(P.q[:l], P.N, 51, 0, 0, 0)
-        y1 = synth.uniform_residues(P.q[:l], P.N, 51, 0, 0, 1)
-        O.relinearize(P, c0, c1, y0, y1, l, seed, b)
-    else:
-        O.keyswitch(P, c0, c1, l, seed, b)
-    return 1
+CPU_BASELINE_WORKLOADS = ("rot1_n16", "relin_n12", "ntt_n16", "rotate_n16", "relin_mul_n12", "relin_mul_n16",
+                          "hoisted8_n16", "batch16_n16", "sweep_n17")
 
 
 def _unit(wl):
+    if wl.name == "ntt_n16":
+        return "limb-NTTs/s"
     return {"rotate": "rotations/s", "hoisted": "rotations/s", "relin": "relinearisations/s"}.get(
         wl.op, "key-switches/s")
 
 
-def cpu_baseline(wl, q, p, budget_s: float = 20.0):
-    """The oracle as it stands, single-threaded, on a bounded sample: as many
-    full operations of the workload as fit in about budget_s seconds."""
-    O, P, b, c0, c1, l, seed = _oracle_inputs(wl, q, p)
-    t0 = time.perf_counter()
-    n = ops = 0
-    while True:
-        ops += oracle_step(wl, O, P, b, c0, c1, l, seed)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s or n >= 50:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": ops / dt, "unit": _unit(wl), "cores": 1, "kind": "oracle",
-            "sample": f"{n} full {wl.op} step(s) ({ops} operation(s)) of {wl.name} (l={l}) in {dt:.1f} s, "
-                      "single thread"}
+class OracleJob:
+    """One operation of a workload on the oracle, with its seeded inputs: a key
+    switch (rotation, relinearisation, hoisted rotations) at the workload's
+    top level, or for the NTT workload a forward + inverse NTT of one limb."""
+
+    def __init__(self, name: str, tag: int = 0):
+        import numpy as np
+        from key_switching_b200 import synth
+        from oracle import oracle as O
+        self.O, self.np = O, np
+        wl = synth.WORKLOADS[name]
+        self.wl = wl
+        P = O.chain(wl.logN, wl.bits, wl.L, wl.alpha)
+        self.P = P
+        prim = [P.prime(g) for g in range(P.L + P.alpha)]
+        self.l = wl.L
+        if name == "ntt_n16":
+            self.x = synth.uniform_residues(prim[:1], P.N, 40, tag)[0]
+            self.q = prim[0]
+            return
+        self.b = np.stack([synth.uniform_residues(prim, P.N, 1, 0xB, j) for j in range(P.dnum)])
+        self.c0 = synth.uniform_residues(P.q[:self.l], P.N, 50, tag, 0, 0)
+        self.c1 = synth.uniform_residues(P.q[:self.l], P.N, 50, tag, 0, 1)
+        self.y0 = synth.uniform_residues(P.q[:self.l], P.N, 51, tag, 0, 0)
+        self.y1 = synth.uniform_residues(P.q[:self.l], P.N, 51, tag, 0, 1)
+        self.seed = synth.chacha_seed(1, tag)
+
+    def run(self) -> int:
+        """Run one operation; returns the number of units done."""
+        O, P, wl, l = self.O, self.P, self.wl, self.l
+        if wl.name == "ntt_n16":
+            y = O.ntt_fwd(self.x, P.logN, self.q)
+            O.ntt_inv(y, P.logN, self.q)
+            return 2
+        if wl.op == "rotate":
+            O.rotate(P, self.c0, self.c1, l, pow(5, 1, 2 * P.N), self.seed, self.b)
+        elif wl.op == "hoisted":
+            gs = [pow(5, 1 << r, 2 * P.N) for r in range(wl.n_rot)]
+            O.rotate_hoisted(P, self.c0, self.c1, l, gs, [self.seed] * wl.n_rot, [self.b] * wl.n_rot)
+            return wl.n_rot
+        elif wl.op == "relin":
+            O.relinearize(P, self.c0, self.c1, self.y0, self.y1, l, self.seed, self.b)
+        else:
+            O.keyswitch(P, self.c0, self.c1, l, self.seed, self.b)
+        return 1
+
+
+def _oracle_worker(name, tag, budget_s, start, q):
+    """A worker process: set up, wait for the others, run whole operations for
+    about budget_s seconds (at least one), report (units, seconds)."""
+    try:
+        job = OracleJob(name, tag)
+        start.wait()
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            n += job.run()
+            dt = time.perf_counter() - t0
+            if dt >= budget_s:
+                break
+        q.put((n, dt))
+    except BaseException as e:  # report, do not hang the parent
+        q.put((0, repr(e)))
+
+
+def oracle_rate(name: str, workers: int, budget_s: float):
+    """Units per second of the oracle on `workers` host processes running
+    independent operations at once: (units summed over the workers) / (the
+    slowest worker's time).  Single-threaded when workers == 1 (in process)."""
+    if workers == 1:
+        job = OracleJob(name)
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            n += job.run()
+            dt = time.perf_counter() - t0
+            if dt >= budget_s:
+                break
+        return n / dt, n, dt
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    start = ctx.Barrier(workers)
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker, args=(name, w, budget_s, start, q)) for w in range(workers)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=600 + 4 * budget_s) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    bad = [r for r in res if not isinstance(r[1], float)]
+    if bad:
+        raise RuntimeError(f"oracle worker failed: {bad[0][1]}")
+    n = sum(r[0] for r in res)
+    dt = max(r[1] for r in res)
+    return n / dt, n, dt
+
+
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def cpu_baseline(name: str, budget_s: float = 10.0):
+    """The oracle as it stands on this host's cores, on bounded samples of the
+    workload: single-threaded, and one independent operation per core on all
+    cores (the headline value); also the two other small workloads named by
+    the survey (N=2^12 key switch, N=2^16 NTT) with the same method."""
+    cores, model = host_cpu()
+    workers = min(cores, 64)
+    from key_switching_b200 import synth
+    wl = synth.WORKLOADS[name]
+    unit = _unit(wl)
+    v1, n1, t1 = oracle_rate(name, 1, budget_s)
+    va, na, ta = oracle_rate(name, workers, budget_s)
+    out = {"value": va, "unit": unit, "cores": workers, "kind": "oracle", "cpu_model": model, "nproc": cores,
+           "sample": f"{na} operation(s) of {name} (top level) on {workers} processes in {ta:.1f} s; "
+                     f"single thread: {n1} in {t1:.1f} s",
+           "single_thread": {"value": v1, "unit": unit, "cores": 1}}
+    others = {}
+    for other in ("relin_n12", "ntt_n16"):
+        if other == name:
+            continue
+        ow = synth.WORKLOADS[other]
+        s1 = oracle_rate(other, 1, budget_s / 4)
+        sa = oracle_rate(other, workers, budget_s / 4)
+        others[other] = {"unit": _unit(ow), "single_thread": s1[0], "all_cores": sa[0], "cores": workers,
+                         "sample": f"{s1[1]} unit(s) in {s1[2]:.1f} s on 1 thread; {sa[1]} in {sa[2]:.1f} s "
+                                   f"on {workers} processes"}
+    out["other_workloads"] = others
+    return out
 
 
 def run_reference(args):
+    """The oracle on the host cores, on this arm's workload, metric and unit:
+    one independent operation per core at a time, each step a bounded sample."""
     world, rank, local = dist_setup()
     if rank != 0:
         return
-    from key_switching_b200 import pc, synth
+    from key_switching_b200 import synth
     wl = synth.WORKLOADS[args.workload]
-    q, p = pc.chain(wl.logN, wl.bits, wl.L, wl.alpha)
-    O, P, b, c0, c1, l, seed = _oracle_inputs(wl, q, p)
-    budget = args.cpu_budget * 6
-    t0 = time.perf_counter()
-    for _ in range(min(args.warmup, 1)):
-        oracle_step(wl, O, P, b, c0, c1, l, seed)
-    t_one = max(1e-3, time.perf_counter() - t0)
-    steps = max(1, min(args.steps, int(budget / t_one)))
-    t0 = time.perf_counter()
-    ops = 0
-    for _ in range(steps):
-        ops += oracle_step(wl, O, P, b, c0, c1, l, seed)
-    dt = time.perf_counter() - t0
-    v = ops / dt
+    cores, model = host_cpu()
+    workers = min(cores, 64)
     unit = _unit(wl)
-    metric = "key-switches/s at N=2^16 (1 B200); achieved HBM GB/s and % of roofline"
-    if wl.op in ("rotate", "hoisted"):
-        metric = (f"rotations/s at N=2^{wl.logN} ({'single' if wl.op == 'rotate' else f'{wl.n_rot} hoisted'}"
-                  " rotation(s) per ciphertext; 1 B200)")
-    elif wl.op == "relin":
-        metric = f"ciphertext products (tensor + relinearisation) per second at N=2^{wl.logN} (1 B200)"
-    elif wl.name == "sweep_n17":
-        metric = "key-switches/s at N=2^17 level sweep 40..1 (1 B200)"
+    # a few seconds per step, the whole run within a few minutes
+    budget = max(2.0, min(12.0, 150.0 / max(1, args.steps)))
+    v, n, dt = oracle_rate(args.workload, workers, budget * max(1, args.steps))
+    metric = workload_metric(wl)
+    sample = (f"{n} unit(s) of {wl.name} (top level) on {workers} processes, one independent operation per "
+              f"process at a time, in {dt:.1f} s ({args.steps} step(s) of ~{budget:.0f} s requested)")
     res = {"impl": "reference", "metric": metric,
-           "value": v, "unit": unit, "n_gpus": 1, "steps": steps, "warmup": min(args.warmup, 1),
-           "ms_per_step": dt * 1e3 / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": "u32", "data": "synthetic",
+           "value": v, "unit": unit, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "u32", "data": "synthetic",
            "config": {"workload": f"{wl.name}: N=2^{wl.logN}, L={wl.L}, alpha={wl.alpha}, dnum={wl.dnum}, "
-                      "1 ct/step at the top level, key a-half regenerated (ChaCha12)"},
-           "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle",
-                            "sample": f"{steps} of {args.steps} requested step(s), each one full {wl.op} "
-                                      f"({ops} operation(s) in all), time-bounded, single thread"},
+                      "operations at the top level, key a-half regenerated (ChaCha12)"},
+           "cpu_baseline": {"value": v, "unit": unit, "cores": workers, "kind": "oracle", "cpu_model": model,
+                            "nproc": cores, "sample": sample},
            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
@@ -566,17 +735,19 @@ def main():
                              "hoisted8_n16", "relin_mul_n12", "relin_mul_n16"])
     ap.add_argument("--keys", default="regen", choices=["regen", "stored"])
     ap.add_argument("--no-graph", action="store_true",
-                    help="call pc_keyswitch every step instead of replaying a CUDA graph of it")
+                    help="call the library every step instead of replaying a CUDA graph of the step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle work per cpu_baseline sample")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
-    else:
-        run_ours(args)
+        return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(sys.argv[1:], args.gpus))
+    run_ours(args)
 
 
 if __name__ == "__main__":

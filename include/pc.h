@@ -49,8 +49,8 @@ extern "C" {
 #define PC_E_ARG (-1)       /* null pointer, level/size out of range, bad params */
 #define PC_E_ALIGN (-2)     /* a device pointer is not 16-byte aligned */
 #define PC_E_CUDA (-3)      /* a CUDA call or launch failed (see pc_strerror) */
-#define PC_E_DEVICE (-4)    /* a kernel reported an error through the device error word */
-#define PC_E_TIMEOUT (-5)   /* a bounded device wait gave up */
+#define PC_E_DEVICE (-4)    /* an input check (pc_set_checks) set the device error word */
+/* (-5) is not used: no call waits on the device with a time limit */
 #define PC_E_PRIME (-6)     /* a modulus is not prime, not = 1 mod 2N, or >= 2^31 */
 #define PC_E_WORKSPACE (-7) /* no workspace set, or smaller than pc_workspace_bytes */
 #define PC_E_TOO_BIG (-8)   /* size beyond the static scratch of pc_modup_noalloc */
@@ -132,15 +132,18 @@ int pc_modup(pc_ctx *ctx, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stre
  * memory (a plugin inside a host framework that owns every device allocation,
  * or a latency-critical path that cannot afford cudaMalloc's device-wide
  * synchronisation).  The pages have no counterpart of this call; it computes
- * exactly what pc_modup computes, with the same arguments, layouts and status
- * codes, and needs no pc_set_workspace.  Its l*N words of scratch live in one
+ * exactly what pc_modup computes, with the same arguments and layouts, and
+ * needs no pc_set_workspace.  Its l*N words of scratch live in one
  * statically allocated device array of 2^21 words (8 MiB) that the library
- * holds on every device it is loaded on until the process exits; l*N above
- * 2^21 returns PC_E_TOO_BIG.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress, with that device current) and caches
- * it, so that first call should be made before any stream capture.  All calls
- * share the array and it keeps the last call's contents (nothing in it needs
- * to start at zero); calls whose kernels overlap on the GPU race on it. */
+ * holds on every device it is loaded on until the process exits.  The
+ * array's device address is looked up once per context, by pc_ctx_create,
+ * with the context's device current (so this call does no lookup and may be
+ * made at any time).  All calls share the array and it keeps the last call's
+ * contents (nothing in it needs to start at zero); calls whose kernels overlap
+ * on the GPU (two streams, or two host threads) race on it, so callers must
+ * order them, e.g. on one stream.  Returns PC_OK, PC_E_ARG, PC_E_ALIGN,
+ * PC_E_TOO_BIG (l*N above 2^21: N=2^16 up to l=32, N=2^17 up to l=16) or
+ * PC_E_CUDA; never PC_E_WORKSPACE. */
 int pc_modup_noalloc(pc_ctx *ctx, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream stream);
 
 /* Key inner product with in-kernel ChaCha12 regeneration of 'a'.
@@ -256,6 +259,35 @@ int pc_rotate_hoisted(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint3
 int pc_relinearize(pc_ctx *ctx, const uint32_t *x, const uint32_t *y, uint32_t l, const pc_ksk *k,
                    uint32_t *out, pc_stream stream);
 
+/* Baby-step giant-step linear transform with hoisted baby steps: the
+ * homomorphic matrix-vector product by the diagonal method that makes up the
+ * CoeffsToSlots and SlotsToCoeffs steps of CKKS bootstrapping.  (Perseus
+ * README, intro: GPT-2 runs 416 bootstraps per token; "Runtime": the `bts`
+ * bootstrap bench of pc-bench; the HEAT listing: bootstraps dominate the
+ * latency.  The pages give no formula, so this is the textbook method:
+ * Halevi-Shoup diagonals split into baby and giant steps, Han-Ki 2020,
+ * Chen-Chillotti-Song 2019.)
+ *   bs_0 = (c0, c1); bs_j = rotation of (c0, c1) by g_baby[j-1], 1 <= j < n1,
+ *          hoisted (one ModUp of c1; as pc_rotate_hoisted)
+ *   W_i  = sum_{j < n1} diag[i][j] (.) bs_j        (slot-wise mod q)
+ *   out  = W_0 + sum_{1 <= i < n2} rotation of W_i by g_giant[i-1]  (as pc_rotate)
+ * diag: device [n2][n1][l][N], NTT-domain plaintexts (the caller's
+ * pre-rotated diagonals), canonical.  g_baby, k_baby: host arrays of n1 - 1
+ * Galois elements and keys (k_baby[j-1] switches s(X^g_baby[j-1]) -> s; all
+ * baby keys regenerate their 'a' halves or all store them, else PC_E_ARG);
+ * g_giant, k_giant: host arrays of n2 - 1 (may be NULL when n1 or n2 is 1).
+ * 1 <= n1, n2 <= PC_BSGS_MAX_STEPS.  c0, c1: device [l][N]; out: device
+ * [2][l][N] (c0' then c1'), not overlapping c0, c1 or diag (PC_E_ARG).  W_i
+ * is never stored: the kernels that read a giant step's input form it from
+ * the baby steps and diagonals, and the last kernel of each giant step adds
+ * its result to out.  Needs a workspace of
+ * pc_linear_transform_workspace_bytes(l, n1), else PC_E_WORKSPACE. */
+#define PC_BSGS_MAX_STEPS 64
+size_t pc_linear_transform_workspace_bytes(const pc_ctx *ctx, uint32_t l, uint32_t n1);
+int pc_linear_transform(pc_ctx *ctx, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t n1,
+                        const uint32_t *g_baby, const pc_ksk *k_baby, uint32_t n2, const uint32_t *g_giant,
+                        const pc_ksk *k_giant, const uint32_t *diag, uint32_t *out, pc_stream stream);
+
 /* Test hook: write the regenerated 'a' words for level l.  a_out: device
  * [beta][l+alpha][N], a_out[j][t][k] = a_{j,g(t)}[k] where (spec v1) block
  * b = k/8 of ChaCha12 with state words (constants "expand 32-byte k", seed as
@@ -264,9 +296,24 @@ int pc_relinearize(pc_ctx *ctx, const uint32_t *x, const uint32_t *y, uint32_t l
 int pc_expand_a(pc_ctx *ctx, const uint8_t seed[32], uint32_t l, uint32_t *a_out,
                 pc_stream stream);
 
+/* Input checks.  With PC_CHECK_INPUTS set, every operation above first runs
+ * a kernel over the residues it reads (ciphertext limbs, accumulators,
+ * extended limbs, both halves of every key) and sets bits of the context's
+ * device error word for residues not below their prime: PC_ERR_INPUT for a
+ * data operand, PC_ERR_KEY for a key half.  The check reads only the buffers
+ * the call reads anyway, never traps, and does not stop the call; pc_check
+ * reports the result.  Off by default (it reads every input once more).
+ * flags: 0 or PC_CHECK_INPUTS, else PC_E_ARG. */
+#define PC_CHECK_INPUTS 1u
+#define PC_ERR_INPUT 1u
+#define PC_ERR_KEY 2u
+int pc_set_checks(pc_ctx *ctx, uint32_t flags);
+
 /* Synchronise the context's device and read its device error word; returns
- * PC_OK, PC_E_DEVICE (and clears the word), or PC_E_CUDA. */
+ * PC_OK, PC_E_DEVICE (the word was set: it is cleared, and its value kept
+ * for pc_last_error_word), or PC_E_CUDA. */
 int pc_check(pc_ctx *ctx);
+uint32_t pc_last_error_word(const pc_ctx *ctx);
 
 /* Human-readable text for a status code (the last CUDA error for PC_E_CUDA). */
 const char *pc_strerror(int code);

@@ -2,7 +2,8 @@
 
     python -m key_switching_b200.build [--force]
 
-Produces key_switching_b200/libpc.so from key_switching_b200/csrc/*.cu.  No GPU
+Produces key_switching_b200/libpc.so from key_switching_b200/csrc/*.cu (the
+kernel file once per ring degree, -DPC_LOGN=10..17, all in parallel).  No GPU
 is needed to build (nvcc cross-compiles).
 """
 from __future__ import annotations
@@ -20,9 +21,12 @@ ROOT = os.path.dirname(HERE)
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "--expt-relaxed-constexpr",
 ]
+
+
+LOGNS = range(10, 18)  # ring degrees 2^10 .. 2^17
 
 
 def nvcc() -> str:
@@ -40,15 +44,42 @@ def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
+    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
+        + glob.glob(os.path.join(CSRC, "*.inc"))
     deps.append(os.path.join(ROOT, "include", "pc.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every csrc/*.cu to an object (in parallel, one nvcc per file)
+    and link them into libpc.so; a no-op when the library is newer than every
+    source."""
     if not force and not needs_build():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *sources()]
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(HERE, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    inc = ["-I", os.path.join(ROOT, "include")]
+
+    def compile_one(src, name, defs):
+        obj = os.path.join(objdir, name + ".o")
+        cmd = [nvcc(), *NVCC_FLAGS, *defs, *inc, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.check_call(cmd)
+        return obj
+
+    # kernels.cu holds every kernel template; it is compiled once per ring
+    # degree (its launchers for degree 2^k live in namespace pc::n<k>)
+    jobs = []
+    for src in sources():
+        if os.path.basename(src) == "kernels.cu":
+            jobs += [(src, f"kernels_n{k}", [f"-DPC_LOGN={k}"]) for k in LOGNS]
+        else:
+            jobs.append((src, os.path.basename(src)[:-3], []))
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
+        objs = list(ex.map(lambda j: compile_one(*j), jobs))
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB + ".tmp", *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)

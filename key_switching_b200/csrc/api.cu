@@ -102,18 +102,7 @@ u32 neg_inv32(u32 u) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-struct DeviceGuard {
-    int prev = -1;
-    bool ok = true;
-    explicit DeviceGuard(int dev) {
-        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
-        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
-    }
-    ~DeviceGuard() {
-        int cur;
-        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-    }
-};
+using pc::DeviceGuard;
 
 // workspace regions for B ciphertexts at level l (words)
 struct Layout {
@@ -158,6 +147,27 @@ void prof_release(pc_ctx *c) {
     delete[] c->prof_ev;
     c->prof_ev = nullptr;
     c->prof_max = c->prof_used = 0;
+}
+
+// PC_CHECK_INPUTS: before a call runs, a kernel checks that every residue
+// it reads is canonical and records a violation in the device error word.
+cudaError_t check_limbs(const pc_ctx *c, const u32 *x, u32 nlimbs, u32 Z, size_t zs, int mode, u32 first,
+                               u32 period, u32 l, int bit, cudaStream_t s) {
+    if (!(c->checks & PC_CHECK_INPUTS) || !x) return cudaSuccess;
+    return pc::launch_check(c, x, nlimbs, Z, zs, mode, first, period, l, bit, s);
+}
+// a ciphertext-like input: Z slices of nlimbs limbs, limb t mod l on q_t
+cudaError_t check_ct(const pc_ctx *c, const u32 *x, u32 nlimbs, u32 l, u32 Z, size_t zs, cudaStream_t s) {
+    return check_limbs(c, x, nlimbs, Z, zs, 1, 0, l, l, PC_ERR_INPUT, s);
+}
+// both halves of n keys ([dnum][L+alpha][N], global prime of limb t = t mod (L+alpha))
+cudaError_t check_keys(const pc_ctx *c, const pc_ksk *k, u32 n, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    for (u32 i = 0; i < n && e == cudaSuccess; ++i) {
+        e = check_limbs(c, k[i].b, c->dnum * c->NP, 1, 0, 2, 0, c->NP, 0, PC_ERR_KEY, s);
+        if (e == cudaSuccess) e = check_limbs(c, k[i].a, c->dnum * c->NP, 1, 0, 2, 0, c->NP, 0, PC_ERR_KEY, s);
+    }
+    return e;
 }
 
 }  // namespace
@@ -375,11 +385,15 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
     T.NP = NP;
     e = pc::prepare_kernels(c);
     if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
+    // the device address of pc_modup_noalloc's static scratch (device current)
+    e = pc::noalloc_setup(c);
+    if (e != cudaSuccess) { cudaFree(blk); delete c; return cuda_fail(e); }
     // Launch attributes.  Programmatic dependent launch lets each kernel stage
-    // its tables while its predecessor drains.  The constant tables are read
-    // by every key switch; an access-policy window marks them persisting in
-    // L2 (within this context's persisting carve-out) so the streamed keys
-    // and ciphertexts do not evict them.
+    // its tables while its predecessor drains.  Opt-in (PC_L2_PERSIST=1 at
+    // context creation): an access-policy window marks the constant tables
+    // persisting in L2 so the streamed keys and ciphertexts do not evict them;
+    // that raises the process's persisting-L2 limit, which other kernels of
+    // the process then share, so it is off unless asked for.
     c->use_pdl = getenv("PC_NO_PDL") ? 0 : 1;
     {
         int lo_pri = 0, hi_pri = 0;
@@ -401,7 +415,8 @@ int pc_ctx_create(const pc_params *P, int device, pc_ctx **out) {
     int max_persist = 0, max_window = 0;
     cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, device);
     cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, device);
-    if (!getenv("PC_NO_L2_PERSIST") && max_persist > 0 && max_window > 0) {
+    const char *l2p = getenv("PC_L2_PERSIST");
+    if (l2p && l2p[0] == '1' && max_persist > 0 && max_window > 0) {
         size_t want = total < (size_t)max_persist ? total : (size_t)max_persist;
         size_t cur = 0;
         cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize);
@@ -472,6 +487,8 @@ int pc_ntt_fwd(pc_ctx *c, uint32_t *x, uint32_t first_prime, uint32_t nlimbs, ui
     DeviceGuard dg(c->device);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t z = (size_t)nlimbs * c->N;
+    if (cudaError_t e = check_limbs(c, x, nlimbs, batch, z, 0, first_prime, nlimbs, 0, PC_ERR_INPUT, s))
+        return cuda_fail(e);
     cudaError_t e = pc::launch_col(c, true, x, x, first_prime, nlimbs, batch, z, z, 0, s);
     if (e == cudaSuccess) e = pc::launch_row(c, true, x, x, first_prime, nlimbs, batch, z, z, true, false, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
@@ -484,6 +501,8 @@ int pc_ntt_inv(pc_ctx *c, uint32_t *x, uint32_t first_prime, uint32_t nlimbs, ui
     DeviceGuard dg(c->device);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t z = (size_t)nlimbs * c->N;
+    if (cudaError_t e = check_limbs(c, x, nlimbs, batch, z, 0, first_prime, nlimbs, 0, PC_ERR_INPUT, s))
+        return cuda_fail(e);
     cudaError_t e = pc::launch_row(c, false, x, x, first_prime, nlimbs, batch, z, z, false, false, s);
     if (e == cudaSuccess) e = pc::launch_col(c, false, x, x, first_prime, nlimbs, batch, z, z, 1, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
@@ -502,7 +521,8 @@ int pc_modup(pc_ctx *c, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream
     cudaStream_t s = (cudaStream_t)stream;
     const Layout Lw = layout(c, l, 1);
     u32 *w1 = (u32 *)c->ws + Lw.w1;
-    cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, true, s);
+    cudaError_t e = check_ct(c, c1, l, l, 1, 0, s);
+    if (e == cudaSuccess) e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, true, s);
     if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, false, s);
     if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
@@ -518,8 +538,12 @@ int pc_keyswitch_inner(pc_ctx *c, const uint32_t *ext, uint32_t l, const pc_ksk 
     kp.b[0] = k->b;
     kp.a[0] = k->a;
     seed_words(k->seed, kp.seed[0]);
-    cudaError_t e = pc::launch_inner(c, false, ext, 0, nullptr, 0, acc, 0, l, kp, 1, k->a == nullptr, false,
-                                     (cudaStream_t)stream);
+    const cudaStream_t s = (cudaStream_t)stream;
+    const u32 beta = (l + c->alpha - 1) / c->alpha, ll = l + c->alpha;
+    cudaError_t e = check_limbs(c, ext, beta * ll, 1, 0, 1, 0, ll, l, PC_ERR_INPUT, s);
+    if (e == cudaSuccess) e = check_keys(c, k, 1, s);
+    if (e == cudaSuccess)
+        e = pc::launch_inner(c, false, ext, 0, nullptr, 0, acc, 0, l, kp, 1, k->a == nullptr, false, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
@@ -532,9 +556,10 @@ int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_str
     const Layout Lw = layout(c, l, 1);
     u32 *wacc = (u32 *)c->ws + Lw.acc, *wu = (u32 *)c->ws + Lw.u;
     const size_t N = c->N, ll = l + c->alpha;
+    cudaError_t e = check_limbs(c, acc, 2 * (u32)ll, 1, 0, 1, 0, (u32)ll, l, PC_ERR_INPUT, s);
     // special-prime limbs of both halves: inverse row pass into the workspace
-    cudaError_t e =
-        pc::launch_row(c, false, acc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, false, true, s);
+    if (e == cudaSuccess)
+        e = pc::launch_row(c, false, acc + l * N, wacc + l * N, c->L, c->alpha, 2, ll * N, ll * N, false, true, s);
     if (e == cudaSuccess) e = pc::launch_colconv(c, 1, wacc, 2 * ll * N, wu, 2 * l * N, l, 1, true, s);
     if (e == cudaSuccess) e = pc::launch_moddown_row(c, wu, 0, acc, 0, nullptr, 0, out, out + l * N, 0, l, 1, s);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
@@ -547,10 +572,14 @@ int pc_moddown(pc_ctx *c, const uint32_t *acc, uint32_t l, uint32_t *out, pc_str
 // and to c0.  mul: c1 is the slot-wise product c1 * mul (relinearisation's
 // d2); rx, ry: the tensor terms d0, d1 of ciphertexts rx, ry are added to the
 // outputs instead of c0.
+// mac: c1 and c0 are halves 1 and 0 of the giant-step operand W of a linear
+// transform (formed from the baby steps and diagonals as they are read), and
+// the results are added to the outputs.
 struct KsInput {
     u32 galois = 1;
     const u32 *hoist = nullptr;
     const u32 *mul = nullptr, *rx = nullptr, *ry = nullptr;
+    const pc::MacIn *mac = nullptr;
 };
 
 // x^-1 mod 2N for odd x (Newton iteration on the 2-adic inverse).
@@ -571,7 +600,7 @@ static cudaEvent_t *profile_slot(pc_ctx *c) {
 
 // c1 is read transformed by the ModUp row kernel, which then stores that
 // transformed copy in the workspace for the inner product's own-digit limbs
-static bool c1_transformed(const KsInput &in) { return in.galois != 1 || in.mul; }
+static bool c1_transformed(const KsInput &in) { return in.galois != 1 || in.mul || in.mac; }
 
 // ModUp up to the column-pass output T in the workspace (laid out for Blay
 // ciphertexts): inverse row pass of c1 (through the input transform), then
@@ -583,7 +612,7 @@ static cudaError_t ks_modup(pc_ctx *c, const u32 *c1, size_t cz, u32 l, u32 B, u
     auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
     mark(0);
     cudaError_t e = pc::launch_row(c, false, c1, ws + Lw.w1, 0, l, B, cz, Lw.w1z, false, true, s, in.galois, in.mul,
-                                   c1_transformed(in) ? ws + Lw.x : nullptr);
+                                   c1_transformed(in) ? ws + Lw.x : nullptr, in.mac);
     mark(1);
     if (e == cudaSuccess) e = pc::launch_colconv(c, 0, ws + Lw.w1, Lw.w1z, ws + Lw.t, Lw.tz, l, B, true, s);
     mark(2);
@@ -654,7 +683,7 @@ static cudaError_t ks_finish(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz,
     const pc::RotPack rp = rotpack(0, B < (u32)pc::KEYS_PER_LAUNCH ? B : (u32)pc::KEYS_PER_LAUNCH);
     if (e == cudaSuccess)
         e = pc::launch_moddown_row(c, wu, Lw.uz, wacc, Lw.accz, in.rx ? nullptr : c0, cz, o0, o1, oz, l, B, s,
-                                   rot ? &rp : nullptr, in.rx, in.ry);
+                                   rot ? &rp : nullptr, in.rx, in.ry, in.mac);
     mark(5);
     return e;
 }
@@ -670,7 +699,14 @@ static int keyswitch_core(pc_ctx *c, const u32 *c0, const u32 *c1, size_t cz, u3
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (profile && cudaStreamIsCapturing(s, &cap) != cudaSuccess) cap = cudaStreamCaptureStatusNone;
     cudaEvent_t *ev = profile && cap == cudaStreamCaptureStatusNone ? profile_slot(c) : nullptr;
-    cudaError_t e = ks_modup(c, c1, cz, l, B, B, in, s, ev);
+    // input checks (PC_CHECK_INPUTS): the ciphertext halves, the second
+    // factor of a product, and the keys
+    cudaError_t e = check_keys(c, keys, B, s);
+    if (e == cudaSuccess && in.rx) e = check_ct(c, in.rx, 2 * l, l, 1, 0, s);
+    if (e == cudaSuccess && in.ry) e = check_ct(c, in.ry, 2 * l, l, 1, 0, s);
+    if (e == cudaSuccess && !in.rx) e = check_ct(c, c1, l, l, B, cz, s);
+    if (e == cudaSuccess && c0) e = check_ct(c, c0, l, l, B, cz, s);
+    if (e == cudaSuccess) e = ks_modup(c, c1, cz, l, B, B, in, s, ev);
     if (e == cudaSuccess) e = ks_finish(c, c0, c1, cz, l, keys, B, B, o0, o1, cz, in, s, ev);
     return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
@@ -821,7 +857,10 @@ int pc_rotate_hoisted(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_
     if (int r = need_ws(c, l, Blay)) return r;
     DeviceGuard dg(c->device);
     const cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = ks_modup(c, c1, 0, l, 1, Blay, KsInput{}, s, nullptr);
+    cudaError_t e = check_keys(c, keys, n, s);
+    if (e == cudaSuccess) e = check_ct(c, c0, l, l, 1, 0, s);
+    if (e == cudaSuccess) e = check_ct(c, c1, l, l, 1, 0, s);
+    if (e == cudaSuccess) e = ks_modup(c, c1, 0, l, 1, Blay, KsInput{}, s, nullptr);
     for (u32 i0 = 0; e == cudaSuccess && i0 < n; i0 += Blay) {
         const u32 nb = n - i0 < Blay ? n - i0 : Blay;
         KsInput in;
@@ -848,6 +887,80 @@ int pc_relinearize(pc_ctx *c, const uint32_t *x, const uint32_t *y, uint32_t l, 
     in.rx = x;
     in.ry = y;
     return keyswitch_core(c, nullptr, x + lN, 0, l, k, 1, out, out + lN, (cudaStream_t)stream, in);
+}
+
+// pc_linear_transform: the key switch's workspace for the hoisted baby steps
+// (up to 16 slices), then the n1 - 1 baby-step outputs [n1-1][2][l][N]
+static u32 lt_slices(u32 n1) { return n1 <= 1 ? 1 : (n1 - 1 < (u32)pc::KEYS_PER_LAUNCH ? n1 - 1 : pc::KEYS_PER_LAUNCH); }
+static size_t lt_ws_words(const pc_ctx *c, u32 l, u32 n1) {
+    return layout(c, l, lt_slices(n1)).total + (size_t)(n1 - 1) * 2 * l * c->N;
+}
+
+size_t pc_linear_transform_workspace_bytes(const pc_ctx *c, uint32_t l, uint32_t n1) {
+    if (!c || l < 1 || l > c->L || n1 < 1 || n1 > PC_BSGS_MAX_STEPS) return 0;
+    return lt_ws_words(c, l, n1) * sizeof(u32);
+}
+
+int pc_linear_transform(pc_ctx *c, const uint32_t *c0, const uint32_t *c1, uint32_t l, uint32_t n1,
+                        const uint32_t *g_baby, const pc_ksk *k_baby, uint32_t n2, const uint32_t *g_giant,
+                        const pc_ksk *k_giant, const uint32_t *diag, uint32_t *out, pc_stream stream) {
+    if (!c || !c0 || !c1 || !diag || !out || l < 1 || l > c->L) return PC_E_ARG;
+    if (n1 < 1 || n2 < 1 || n1 > PC_BSGS_MAX_STEPS || n2 > PC_BSGS_MAX_STEPS) return PC_E_ARG;
+    if ((n1 > 1 && (!g_baby || !k_baby)) || (n2 > 1 && (!g_giant || !k_giant))) return PC_E_ARG;
+    for (u32 j = 0; j + 1 < n1; ++j) {
+        if (!galois_ok(c, g_baby[j])) return PC_E_ARG;
+        if (int r = check_ksk(c, &k_baby[j])) return r;
+        if ((k_baby[j].a == nullptr) != (k_baby[0].a == nullptr)) return PC_E_ARG;  // one key mode per batch
+    }
+    for (u32 i = 0; i + 1 < n2; ++i) {
+        if (!galois_ok(c, g_giant[i])) return PC_E_ARG;
+        if (int r = check_ksk(c, &k_giant[i])) return r;
+    }
+    if (!aligned16(c0) || !aligned16(c1) || !aligned16(diag) || !aligned16(out)) return PC_E_ALIGN;
+    const size_t lN = (size_t)l * c->N, b1 = lN * sizeof(u32);
+    if (overlaps(out, 2 * b1, c0, b1) || overlaps(out, 2 * b1, c1, b1) ||
+        overlaps(out, 2 * b1, diag, (size_t)n1 * n2 * b1))
+        return PC_E_ARG;
+    if (!c->ws || c->ws_bytes < lt_ws_words(c, l, n1) * sizeof(u32)) return PC_E_WORKSPACE;
+    DeviceGuard dg(c->device);
+    const cudaStream_t s = (cudaStream_t)stream;
+    const u32 Blay = lt_slices(n1);
+    u32 *bs = (u32 *)c->ws + layout(c, l, Blay).total;
+    cudaError_t e = check_keys(c, k_baby, n1 - 1, s);
+    if (e == cudaSuccess) e = check_keys(c, k_giant, n2 - 1, s);
+    if (e == cudaSuccess) e = check_ct(c, c0, l, l, 1, 0, s);
+    if (e == cudaSuccess) e = check_ct(c, c1, l, l, 1, 0, s);
+    if (e == cudaSuccess) e = check_ct(c, diag, l, l, n1 * n2, lN, s);
+    // baby steps: hoisted rotations of (c0, c1), one ModUp
+    if (e == cudaSuccess && n1 > 1) e = ks_modup(c, c1, 0, l, 1, Blay, KsInput{}, s, nullptr);
+    for (u32 j0 = 0; e == cudaSuccess && j0 + 1 < n1; j0 += Blay) {
+        const u32 nb = n1 - 1 - j0 < Blay ? n1 - 1 - j0 : Blay;
+        KsInput in;
+        in.hoist = g_baby + j0;
+        u32 *o = bs + 2 * (size_t)j0 * lN;
+        e = ks_finish(c, c0, c1, 0, l, k_baby + j0, nb, Blay, o, o + lN, 2 * lN, in, s, nullptr);
+    }
+    // giant step 0: out = sum_j d_0j (.) bs_j; giant step i >= 1: out += the
+    // rotation of W_i = sum_j d_ij (.) bs_j, W_i formed as the kernels read it
+    pc::MacIn m{};
+    m.x0[0] = c0;
+    m.x0[1] = c1;
+    m.xs = bs;
+    m.xz = 2 * lN;
+    m.hz = lN;
+    m.d = diag;
+    m.dz = lN;
+    m.n1 = n1;
+    if (e == cudaSuccess) e = pc::launch_mac(c, m, l, out, s);
+    for (u32 i = 1; e == cudaSuccess && i < n2; ++i) {
+        m.d = diag + (size_t)i * n1 * lN;
+        KsInput in;
+        in.galois = g_giant[i - 1];
+        in.mac = &m;
+        e = ks_modup(c, c1, 0, l, 1, 1, in, s, nullptr);
+        if (e == cudaSuccess) e = ks_finish(c, c0, c1, 0, l, &k_giant[i - 1], 1, 1, out, out + lN, 0, in, s, nullptr);
+    }
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
 }
 
 int pc_keyswitch_host(pc_ctx *c, const uint32_t *ct, uint32_t n, uint32_t l, const pc_ksk *keys, uint32_t *out,
@@ -955,9 +1068,19 @@ int pc_check(pc_ctx *c) {
     e = cudaMemcpy(&word, c->tab.err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e);
     if (word) {
-        cudaMemset(c->tab.err, 0, sizeof(int));
+        c->last_err_word = (uint32_t)word;
+        e = cudaMemset(c->tab.err, 0, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
         return PC_E_DEVICE;
     }
+    return PC_OK;
+}
+
+uint32_t pc_last_error_word(const pc_ctx *c) { return c ? c->last_err_word : 0; }
+
+int pc_set_checks(pc_ctx *c, uint32_t flags) {
+    if (!c || (flags & ~(uint32_t)PC_CHECK_INPUTS)) return PC_E_ARG;
+    c->checks = flags;
     return PC_OK;
 }
 
@@ -967,8 +1090,7 @@ const char *pc_strerror(int code) {
         case PC_E_ARG: return "invalid argument (null pointer, level or size out of range, bad parameters)";
         case PC_E_ALIGN: return "device pointer not 16-byte aligned (workspace: 256-byte)";
         case PC_E_CUDA: return cudaGetErrorString(g_last_cuda);
-        case PC_E_DEVICE: return "a kernel reported an error through the device error word";
-        case PC_E_TIMEOUT: return "a bounded device wait gave up";
+        case PC_E_DEVICE: return "an input check found a residue not below its prime (device error word set)";
         case PC_E_PRIME: return "modulus not prime, not 1 mod 2N, repeated, or >= 2^31";
         case PC_E_WORKSPACE: return "workspace missing or smaller than pc_workspace_bytes";
         case PC_E_TOO_BIG: return "l*N exceeds the static scratch of pc_modup_noalloc (2^21 words)";

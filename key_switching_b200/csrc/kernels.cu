@@ -30,6 +30,7 @@
 
 #include "chacha.cuh"
 #include "ntt.cuh"
+#include "launch.cuh"
 #include "pc_internal.h"
 
 namespace pc {
@@ -38,8 +39,18 @@ namespace pc {
 // ptxas fits the kernels into 32 registers (full occupancy); these
 // latency-bound kernels run faster with the registers they naturally use
 // (48-105), which keep more independent loads and butterflies in flight.
-constexpr int ROW_MIN_CTAS = 8;
-constexpr int COLCONV_MIN_CTAS = 1;
+#ifndef PC_ROW_MIN_CTAS
+#define PC_ROW_MIN_CTAS 8
+#endif
+#ifndef PC_COLCONV_MIN_CTAS
+#define PC_COLCONV_MIN_CTAS 1
+#endif
+#ifndef PC_INNER_MIN_CTAS
+#define PC_INNER_MIN_CTAS 4
+#endif
+constexpr int ROW_MIN_CTAS = PC_ROW_MIN_CTAS;
+constexpr int COLCONV_MIN_CTAS = PC_COLCONV_MIN_CTAS;
+constexpr int INNER_MIN_CTAS = PC_INNER_MIN_CTAS;
 
 // ------------------------------------------------------------------ helpers
 
@@ -130,6 +141,35 @@ __device__ __forceinline__ void load_row_in(u32 v[16], const u32 *x, const u32 *
         }
     }
 }
+// Elements x_of(lt, r) (layout PH) of row `row` of limb `limb` of half h of
+// the giant-step operand W = sum_j d_j (.) bs_j (MacIn), read through
+// X -> X^g: 64-bit sums of the products, folded before each product after the
+// second, one reduction.  Inputs canonical; output canonical.
+template <class PH, int LOGN, int C>
+__device__ __forceinline__ void load_row_mac(u32 v[16], const MacIn &m, int h, u32 limb, int row, int lt, u32 g,
+                                             const PrimeK &pk) {
+    const size_t lo = (size_t)limb << LOGN;
+    u32 k[16];
+    u64 acc[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const u32 x = (u32)(row * C + PH::x_of(lt, r));
+        k[r] = g == 1 ? x : auto_src<LOGN>(x, g);
+        acc[r] = (u64)__ldg(m.d + lo + k[r]) * __ldg(m.x0[h] + lo + k[r]);
+    }
+    for (u32 j = 1; j < m.n1; ++j) {
+        const u32 *dj = m.d + j * m.dz + lo;
+        const u32 *xj = m.xs + (j - 1) * m.xz + h * m.hz + lo;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            if (j >= 2) acc[r] = fold64(acc[r], pk.q, pk.q1s);
+            acc[r] += (u64)__ldg(dj + k[r]) * __ldg(xj + k[r]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) v[r] = shoup(redc64(acc[r], pk.q, pk.qn, pk.q1s), pk.r32, pk.r32s, pk.q);
+}
+
 template <int W>
 struct ColAddr {
     int c;
@@ -192,15 +232,16 @@ constexpr size_t row_smem_bytes(int tiles) {
 // ------------------------------------------------------------------ row pass
 // grid (ROW_BLOCKS, nlimbs, Z).  Row-major limbs in.  Out: row-major (in
 // place allowed), or for CMOUT (inverse only) column-major limbs.
-template <int LOGN, bool FWD, bool CMOUT>
+template <int LOGN, bool FWD, bool CMOUT, bool MAC = false>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int canonical, u32 galois,
-      const u32 *mul, u32 *xout) {
+      const u32 *mul, u32 *xout, MacIn mac) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
     using PLAST = typename LastPhase<GE::LOGC>::type;
     static_assert(!(CMOUT && FWD), "column-major output is for the inverse pass");
+    static_assert(!(MAC && FWD), "the giant-step operand is read by the inverse pass");
     extern __shared__ __align__(16) u32 dyn[];
     uint2 *stw = reinterpret_cast<uint2 *>(dyn);  // [NL][C]
     u32 *sm = dyn + 2 * GE::NL * GE::C;             // [NL][ROW_LS]
@@ -224,7 +265,9 @@ k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
     if constexpr (FWD) {
         gload<PF>(v, src + (size_t)row * GE::C, lt);
     } else {
-        load_row_in<PLAST, LOGN, GE::C>(v, src, mul ? mul + blockIdx.z * zin + limb : nullptr, row, lt, galois, pk);
+        // (MAC: a giant step's operand, half 1, formed from the baby steps)
+        if constexpr (MAC) load_row_mac<PLAST, LOGN, GE::C>(v, mac, 1, blockIdx.y, row, lt, galois, pk);
+        else load_row_in<PLAST, LOGN, GE::C>(v, src, mul ? mul + blockIdx.z * zin + limb : nullptr, row, lt, galois, pk);
         // the transformed input itself (row-major, stride zout) for later readers
         if (xout) gstore<PLAST>(v, xout + blockIdx.z * zout + limb + (size_t)row * GE::C, lt);
     }
@@ -440,7 +483,7 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
 // the shared body, ptxas scheduled the plain kernel's loads later (twice the
 // long-scoreboard stalls at the same instruction count; 84 instead of 80 us
 // at N=2^16, l=24).
-enum { XF_PLAIN = 0, XF_GATHER = 1, XF_MUL = 3 };  // input modes of the ModDown finish
+enum { XF_PLAIN = 0, XF_GATHER = 1, XF_MUL = 3, XF_MAC = 4 };  // input modes of the ModDown finish
 template <int LOGN, bool FUSED, bool REGEN, bool ROT>
 __device__ __forceinline__ void inner_body(const Tables &T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
                                            u32 *acc, size_t accz, u32 l, const KeyPack &kp, int pintt, u32 t0,
@@ -633,7 +676,7 @@ __device__ __forceinline__ void inner_body(const Tables &T, const u32 *src, size
 }
 
 template <int LOGN, bool FUSED, bool REGEN>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 4)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, INNER_MIN_CTAS)
 k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz,
         u32 l, KeyPack kp, int pintt, u32 t0) {
     using GE = Geo<LOGN>;
@@ -798,7 +841,7 @@ __device__ __forceinline__ u32 pick(const u32 (&a)[KEYS_PER_LAUNCH], u32 z) {
 }
 
 template <int LOGN, bool REGEN>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, 4)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, INNER_MIN_CTAS)
 k_inner_rot(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
             KeyPack kp, int pintt, u32 t0, RotPack rp) {
     inner_body<LOGN, true, REGEN, true>(T, src, srcz, c1, c1z, acc, accz, l, kp, pintt, t0,
@@ -811,12 +854,15 @@ k_inner_rot(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u3
 // and d1 (h = 1) of ciphertexts rx, ry ([2][l][N], Z = 1) when rx is given;
 // U column-major, the rest row-major.  out0/out1 may alias c0 only for
 // XF_PLAIN.
-// XF: XF_PLAIN, XF_GATHER (c0 of slice z read through X -> X^rp.galois[z])
-// or XF_MUL (the tensor terms of rx, ry added instead of c0).
+// XF: XF_PLAIN, XF_GATHER (c0 of slice z read through X -> X^rp.galois[z]),
+// XF_MUL (the tensor terms of rx, ry added instead of c0) or XF_MAC (Z = 1:
+// half 0 of the giant-step operand of mac, read through X -> X^rp.galois[0],
+// added instead of c0, and both results added to out0 / out1 in place).
 template <int LOGN, int XF>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
-              size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, RotPack rp, const u32 *rx, const u32 *ry) {
+              size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, RotPack rp, const u32 *rx, const u32 *ry,
+              MacIn mac) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -871,6 +917,16 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
                     cc[r] = shoup(redc64(d, q, pk.qn, pk.q1s), pk.r32, pk.r32s, q);
                 }
             }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) o[r] = red1(o[r] + cc[r], q);
+        } else if constexpr (XF == XF_MAC) {
+            u32 cc[16];
+            if (h == 0) {
+                load_row_mac<PLAST, LOGN, GE::C>(cc, mac, 0, i, row, lt, rp.galois[0], pk);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) o[r] = red1(o[r] + cc[r], q);
+            }
+            gload<PLAST>(cc, (h == 0 ? out0 : out1) + (size_t)i * GE::N + rowoff, lt);
 #pragma unroll
             for (int r = 0; r < 16; ++r) o[r] = red1(o[r] + cc[r], q);
         } else if (h == 0 && c0) {
@@ -957,64 +1013,19 @@ __global__ void k_expand(Tables T, KeyPack kp, u32 l, u32 *out) {
 
 // ================================================================ launchers
 
-#define PC_DISPATCH(LOGN_VAR, ...)                     \
-    switch (LOGN_VAR) {                                \
-        case 10: { constexpr int LG = 10; __VA_ARGS__; break; } \
-        case 11: { constexpr int LG = 11; __VA_ARGS__; break; } \
-        case 12: { constexpr int LG = 12; __VA_ARGS__; break; } \
-        case 13: { constexpr int LG = 13; __VA_ARGS__; break; } \
-        case 14: { constexpr int LG = 14; __VA_ARGS__; break; } \
-        case 15: { constexpr int LG = 15; __VA_ARGS__; break; } \
-        case 16: { constexpr int LG = 16; __VA_ARGS__; break; } \
-        case 17: { constexpr int LG = 17; __VA_ARGS__; break; } \
-        default: return cudaErrorInvalidValue;         \
-    }
+// This file is compiled once per ring degree, with -DPC_LOGN=10..17; its
+// launchers live in namespace pc::n<PC_LOGN> (dispatch.cu picks the one of a
+// context's ring degree), so every kernel template is instantiated for one
+// ring degree per translation unit.
+#ifndef PC_LOGN
+#error "compile kernels.cu with -DPC_LOGN=<log2 of the ring degree>"
+#endif
+#define PC_DISPATCH(LOGN_VAR, ...) { constexpr int LG = PC_LOGN; __VA_ARGS__; }
+#define PC_NS_CAT2(a, b) a##b
+#define PC_NS_CAT(a, b) PC_NS_CAT2(a, b)
+#define PC_NS PC_NS_CAT(n, PC_LOGN)
 
-// Every launch goes through cudaLaunchKernelEx with programmatic stream
-// serialisation (the kernels call pdl_wait before touching data) and, when the
-// context has one, an L2 access-policy window that keeps the constant tables
-// persisting in L2 while the streamed operands pass through.
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_exc(const pc_ctx *c, unsigned cluster_x, void (*kern)(KArgs...), dim3 grid, dim3 block,
-                              size_t smem, cudaStream_t s, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[3];
-    unsigned n = 0;
-    if (cluster_x > 1) {
-        attr[n].id = cudaLaunchAttributeClusterDimension;
-        attr[n].val.clusterDim.x = cluster_x;
-        attr[n].val.clusterDim.y = 1;
-        attr[n].val.clusterDim.z = 1;
-        ++n;
-    }
-    if (c->use_pdl) {
-        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[n].val.programmaticStreamSerializationAllowed = 1;
-        ++n;
-    }
-    if (c->l2_window_bytes) {
-        attr[n].id = cudaLaunchAttributeAccessPolicyWindow;
-        attr[n].val.accessPolicyWindow.base_ptr = c->l2_window_base;
-        attr[n].val.accessPolicyWindow.num_bytes = c->l2_window_bytes;
-        attr[n].val.accessPolicyWindow.hitRatio = c->l2_hit_ratio;
-        attr[n].val.accessPolicyWindow.hitProp = cudaAccessPropertyPersisting;
-        attr[n].val.accessPolicyWindow.missProp = cudaAccessPropertyStreaming;
-        ++n;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = n;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_ex(const pc_ctx *c, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                             cudaStream_t s, Args... args) {
-    return launch_exc(c, 1, kern, grid, block, smem, s, args...);
-}
+namespace PC_NS {
 
 // shared memory of k_colconv: alpha y tiles and one exchange line per warp
 template <class GE>
@@ -1039,6 +1050,7 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
         cudaError_t e = allow_smem(k_row<LG, true, false>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_row<LG, false, false>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_row<LG, false, true>, row_smem_bytes<GE>(1));
+        if (e == cudaSuccess) e = allow_smem(k_row<LG, false, true, true>, row_smem_bytes<GE>(1));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, true>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, false>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, row_smem_bytes<GE>(2));
@@ -1048,6 +1060,7 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
         if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_PLAIN>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_GATHER>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_MUL>, row_smem_bytes<GE>(2));
+        if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_MAC>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_modup_finish<LG>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_colconv<LG, true>, colconv_smem<GE>(c));
         if (e == cudaSuccess) e = allow_smem(k_colconv<LG, false>, colconv_smem<GE>(c));
@@ -1058,20 +1071,21 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
 
 cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
                        size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s, u32 galois,
-                       const u32 *mul, u32 *xout) {
+                       const u32 *mul, u32 *xout, const MacIn *mac) {
+    if (mac && (fwd || !cm_out || Z != 1 || first_prime != 0)) return cudaErrorInvalidValue;
+    const MacIn m = mac ? *mac : MacIn{};
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         dim3 grid(GE::ROW_BLOCKS, nlimbs, Z);
-        if (fwd)
-            e = launch_ex(c, k_row<LG, true, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab,
-                          in, out, first_prime, zin, zout, (int)canonical, galois, mul, xout);
-        else if (cm_out)
-            e = launch_ex(c, k_row<LG, false, true>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(1), s, c->tab,
-                          in, out, first_prime, zin, zout, (int)canonical, galois, mul, xout);
-        else
-            e = launch_ex(c, k_row<LG, false, false>, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(0), s, c->tab,
-                          in, out, first_prime, zin, zout, (int)canonical, galois, mul, xout);
+        auto go = [&](auto kern, int tiles) {
+            return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(tiles), s, c->tab, in, out,
+                             first_prime, zin, zout, (int)canonical, galois, mul, xout, m);
+        };
+        if (fwd) e = go(k_row<LG, true, false>, 0);
+        else if (mac) e = go(k_row<LG, false, true, true>, 1);
+        else if (cm_out) e = go(k_row<LG, false, true>, 1);
+        else e = go(k_row<LG, false, false>, 0);
     });
     return e;
 }
@@ -1137,8 +1151,10 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
 
 cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
                                size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s,
-                               const RotPack *rot, const u32 *rx, const u32 *ry) {
+                               const RotPack *rot, const u32 *rx, const u32 *ry, const MacIn *mac) {
     if (rot && Z > (u32)KEYS_PER_LAUNCH) return cudaErrorInvalidValue;
+    if (mac && (Z != 1 || rx)) return cudaErrorInvalidValue;
+    const MacIn m = mac ? *mac : MacIn{};
     RotPack rp{};
     for (int z = 0; z < KEYS_PER_LAUNCH; ++z) rp.galois[z] = rp.ginv[z] = 1;
     if (rot) rp = *rot;
@@ -1148,9 +1164,10 @@ cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u
         dim3 grid(GE::ROW_BLOCKS, l, Z);
         auto go = [&](auto kern) {
             return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), row_smem_bytes<GE>(2), s, c->tab, U, Uz, acc,
-                             accz, c0, c0z, out0, out1, outz, l, rp, rx, ry);
+                             accz, c0, c0z, out0, out1, outz, l, rp, rx, ry, m);
         };
-        if (rx) e = Z == 1 && ry ? go(k_moddown_row<LG, XF_MUL>) : cudaErrorInvalidValue;
+        if (mac) e = go(k_moddown_row<LG, XF_MAC>);
+        else if (rx) e = Z == 1 && ry ? go(k_moddown_row<LG, XF_MUL>) : cudaErrorInvalidValue;
         else if (rot) e = go(k_moddown_row<LG, XF_GATHER>);
         else e = go(k_moddown_row<LG, XF_PLAIN>);
     });
@@ -1179,4 +1196,5 @@ cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, c
     return e;
 }
 
+}  // namespace n<PC_LOGN>
 }  // namespace pc

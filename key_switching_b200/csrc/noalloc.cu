@@ -11,64 +11,49 @@
 // The array is a file-scope __device__ variable of PC_NOALLOC_SCRATCH_WORDS
 // 32-bit words (8 MiB): every GPU on which the library is loaded holds it
 // until the process exits.  Host code cannot use the variable's name as a
-// device address, so the address is looked up once per device with
-// cudaGetSymbolAddress (on the first call made on that device, with that
-// device current) and cached.  Every call shares the one array and it keeps
+// device address (in host code it names a host-side stand-in), so
+// pc_ctx_create looks the address up once per context, with the context's
+// device current, through noalloc_setup below, and the entry point passes
+// that address to the kernels.  Every call shares the one array and it keeps
 // the previous call's contents; calls whose kernels overlap on the GPU (two
 // streams, or two host threads) race on it.  Nothing in it needs clearing:
 // each call overwrites the l*N words it reads.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "pc_internal.h"
 
 namespace {
-
 constexpr size_t PC_NOALLOC_SCRATCH_WORDS = (size_t)1 << 21;  // 8 MiB
-constexpr int MAX_DEVICES = 128;
-
 }  // namespace
 
 static __device__ __align__(256) uint32_t pc_noalloc_scratch[PC_NOALLOC_SCRATCH_WORDS];
 
-namespace {
+namespace pc {
 
-std::mutex g_scratch_mu;
-void *g_scratch_addr[MAX_DEVICES];
-
-// Device address of pc_noalloc_scratch on `dev` (which must be current).
-int scratch_address(int dev, uint32_t **out) {
-    if (dev < 0 || dev >= MAX_DEVICES) return PC_E_ARG;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, pc_noalloc_scratch);
-        if (e != cudaSuccess || !p) return pc::record_cuda_error(e == cudaSuccess ? cudaErrorUnknown : e);
-        g_scratch_addr[dev] = p;
-    }
-    *out = static_cast<uint32_t *>(g_scratch_addr[dev]);
-    return PC_OK;
+cudaError_t noalloc_setup(pc_ctx *c) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, pc_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    if (!p) return cudaErrorInvalidSymbol;
+    c->noalloc_scratch = static_cast<uint32_t *>(p);
+    return cudaSuccess;
 }
 
-}  // namespace
+}  // namespace pc
 
 extern "C" int pc_modup_noalloc(pc_ctx *c, const uint32_t *c1, uint32_t l, uint32_t *ext, pc_stream stream) {
     if (!c || !c1 || !ext || l < 1 || l > c->L) return PC_E_ARG;
     if ((((uintptr_t)c1) | ((uintptr_t)ext)) & 15u) return PC_E_ALIGN;
     if ((size_t)l * c->N > PC_NOALLOC_SCRATCH_WORDS) return PC_E_TOO_BIG;
-    int prev = -1;
-    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
-    if (prev != c->device && cudaSetDevice(c->device) != cudaSuccess) return pc::record_cuda_error(cudaGetLastError());
-    uint32_t *w1 = nullptr;
-    int rc = scratch_address(c->device, &w1);
-    if (rc == PC_OK) {
-        const cudaStream_t s = (cudaStream_t)stream;
-        cudaError_t e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, true, s);
-        if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, false, s);
-        if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
-        if (e != cudaSuccess) rc = pc::record_cuda_error(e);
-    }
-    if (prev >= 0 && prev != c->device) cudaSetDevice(prev);
-    return rc;
+    if (!c->noalloc_scratch) return PC_E_ARG;
+    pc::DeviceGuard dg(c->device);
+    if (!dg.ok) return pc::record_cuda_error(cudaGetLastError());
+    uint32_t *w1 = c->noalloc_scratch;
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (c->checks & PC_CHECK_INPUTS) e = pc::launch_check(c, c1, l, 1, 0, 1, 0, l, l, PC_ERR_INPUT, s);
+    if (e == cudaSuccess) e = pc::launch_row(c, false, c1, w1, 0, l, 1, 0, 0, false, true, s);
+    if (e == cudaSuccess) e = pc::launch_colconv(c, 0, w1, 0, ext, 0, l, 1, false, s);
+    if (e == cudaSuccess) e = pc::launch_modup_finish(c, c1, ext, l, s);
+    return e == cudaSuccess ? PC_OK : pc::record_cuda_error(e);
 }

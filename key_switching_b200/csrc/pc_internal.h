@@ -57,6 +57,19 @@ struct RotPack {
     u32 ginv[KEYS_PER_LAUNCH];
 };
 
+// Operand of a giant step of a baby-step giant-step linear transform: half h
+// of W = sum_{j < n1} d_j (.) bs_j (slot-wise mod q), where bs_0 is the input
+// ciphertext (half h at x0[h]), baby step j >= 1 has half h at
+// xs + (j-1) xz + h hz, and diagonal j is at d + j dz; limb i of each at + i N.
+struct MacIn {
+    const u32 *x0[2];
+    const u32 *xs;
+    size_t xz, hz;
+    const u32 *d;
+    size_t dz;
+    u32 n1;
+};
+
 }  // namespace pc
 
 struct pc_ctx {
@@ -70,6 +83,12 @@ struct pc_ctx {
     size_t dev_bytes;
     void *ws;         // caller's workspace
     size_t ws_bytes;
+    // device address of the static scratch array of pc_modup_noalloc on
+    // this context's device (looked up at context creation)
+    uint32_t *noalloc_scratch;
+    // PC_CHECK_* flags of pc_set_checks: validate inputs on the device
+    uint32_t checks;
+    uint32_t last_err_word;  // the error word pc_check last found set
     // launch attributes: programmatic dependent launch, L2 persistence of the tables
     int use_pdl;
     void *l2_window_base;
@@ -99,9 +118,11 @@ namespace pc {
 // The inverse pass can read its input limbs through X -> X^galois and / or
 // times the limbs of `mul` (same strides), and store that transformed input
 // (row-major, stride zout) to xout.
+// With mac (inverse, Z = 1): the input limbs are half 1 of the giant-step
+// operand W of *mac (see MacIn) instead of `in`, read through X -> X^galois.
 cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
                        size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s, u32 galois = 1,
-                       const u32 *mul = nullptr, u32 *xout = nullptr);
+                       const u32 *mul = nullptr, u32 *xout = nullptr, const MacIn *mac = nullptr);
 // scale_mode: 0 none (lazy), 1 N^-1 (canonical)
 cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
                        size_t zin, size_t zout, int scale_mode, cudaStream_t s);
@@ -120,12 +141,45 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
                          cudaStream_t s, u32 t0 = 0, u32 nt = 0, const RotPack *rot = nullptr);
 // ModDown finish; c0 of slice z read through X -> X^galois[z] when rot is
 // given, or (rx, ry given) the tensor terms d0, d1 of ciphertexts rx, ry
-// added instead of c0.
+// added instead of c0, or (mac given, Z = 1) half 0 of the giant-step operand
+// W of *mac read through X -> X^galois[0] instead of c0, and the result added
+// to the outputs' previous contents.
 cudaError_t launch_moddown_row(const pc_ctx *c, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
                                size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, u32 Z, cudaStream_t s,
-                               const RotPack *rot = nullptr, const u32 *rx = nullptr, const u32 *ry = nullptr);
+                               const RotPack *rot = nullptr, const u32 *rx = nullptr, const u32 *ry = nullptr,
+                               const MacIn *mac = nullptr);
+// out[h][i] = sum_j d_j (.) bs_j half h (the giant step without rotation),
+// out: [2][l][N] canonical.
+cudaError_t launch_mac(const pc_ctx *c, const MacIn &m, u32 l, u32 *out, cudaStream_t s);
 cudaError_t launch_modup_finish(const pc_ctx *c, const u32 *c1, u32 *ext, u32 l, cudaStream_t s);
 cudaError_t launch_expand(const pc_ctx *c, const u32 seed[8], u32 l, u32 *out, cudaStream_t s);
+// Input validation: OR `bit` into the device error word if any residue of
+// x is not below its prime.  x holds Z slices (stride zs words) of nlimbs
+// limbs of N words; limb t uses prime: mode 0, global index first + t;
+// mode 1, the local limb (t mod period) at level l; mode 2, the global index
+// t mod period (a key half [dnum][L+alpha][N]).
+cudaError_t launch_check(const pc_ctx *c, const u32 *x, u32 nlimbs, u32 Z, size_t zs, int mode, u32 first,
+                         u32 period, u32 l, int bit, cudaStream_t s);
+// Look up the device address of pc_modup_noalloc's static scratch array on
+// the context's device (which must be current) into c->noalloc_scratch.
+cudaError_t noalloc_setup(pc_ctx *c);
+
+// Make `dev` the current device for the lifetime of the guard, then restore
+// the caller's device.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+    DeviceGuard(const DeviceGuard &) = delete;
+    DeviceGuard &operator=(const DeviceGuard &) = delete;
+};
 cudaError_t prepare_kernels(const pc_ctx *c);
 
 // Remember a CUDA error for pc_strerror(PC_E_CUDA); returns PC_E_CUDA.

@@ -16,7 +16,9 @@ LIB_PATH = os.path.join(_HERE, "libpc.so")
 
 PC_OK = 0
 ERRORS = {-1: "PC_E_ARG", -2: "PC_E_ALIGN", -3: "PC_E_CUDA", -4: "PC_E_DEVICE",
-          -5: "PC_E_TIMEOUT", -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE", -8: "PC_E_TOO_BIG"}
+          -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE", -8: "PC_E_TOO_BIG"}
+CHECK_INPUTS = 1           # pc_set_checks flag
+ERR_INPUT, ERR_KEY = 1, 2  # bits of the device error word
 
 # names of every exported entry point of include/pc.h
 EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_workspace_bytes",
@@ -24,7 +26,8 @@ EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_wor
            "pc_moddown", "pc_keyswitch", "pc_keyswitch_batch", "pc_expand_a", "pc_check",
            "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc",
            "pc_rotate", "pc_rotate_hoisted", "pc_relinearize", "pc_keyswitch_host", "pc_host_workspace_bytes",
-           "pc_keyswitch_capture", "pc_graph_launch", "pc_graph_destroy", "pc_capture_begin", "pc_capture_end")
+           "pc_keyswitch_capture", "pc_graph_launch", "pc_graph_destroy", "pc_capture_begin", "pc_capture_end",
+           "pc_set_checks", "pc_last_error_word", "pc_linear_transform", "pc_linear_transform_workspace_bytes")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
 
 
@@ -101,10 +104,19 @@ def lib():
         L.pc_capture_begin.restype = i32
         L.pc_capture_end.argtypes = [vp, ctypes.POINTER(vp)]
         L.pc_capture_end.restype = i32
+        L.pc_linear_transform.argtypes = [vp, vp, vp, u32, u32, ctypes.POINTER(u32), ctypes.POINTER(_Ksk), u32,
+                                          ctypes.POINTER(u32), ctypes.POINTER(_Ksk), vp, vp, vp]
+        L.pc_linear_transform.restype = i32
+        L.pc_linear_transform_workspace_bytes.argtypes = [vp, u32, u32]
+        L.pc_linear_transform_workspace_bytes.restype = sz
         L.pc_expand_a.argtypes = [vp, ctypes.c_char_p, u32, vp, vp]
         L.pc_expand_a.restype = i32
         L.pc_check.argtypes = [vp]
         L.pc_check.restype = i32
+        L.pc_set_checks.argtypes = [vp, u32]
+        L.pc_set_checks.restype = i32
+        L.pc_last_error_word.argtypes = [vp]
+        L.pc_last_error_word.restype = u32
         L.pc_strerror.argtypes = [i32]
         L.pc_strerror.restype = ctypes.c_char_p
         L.pc_microbench.argtypes = [i32, i32, u32, ctypes.POINTER(ctypes.c_double)]
@@ -357,11 +369,42 @@ class Context:
         _ok(lib().pc_relinearize(self._h, _ptr(x), _ptr(y), l, ctypes.byref(k), _ptr(out), _stream(stream)),
             "pc_relinearize")
 
+    def linear_transform_workspace_bytes(self, l: int, n1: int) -> int:
+        return int(lib().pc_linear_transform_workspace_bytes(self._h, l, n1))
+
+    def ensure_linear_transform_workspace(self, l: int, n1: int):
+        """Allocate (with torch) and set a workspace big enough for a linear transform with n1 baby steps."""
+        import torch
+        need = self.linear_transform_workspace_bytes(l, n1)
+        if self._ws is None or self._ws.numel() * self._ws.element_size() < need:
+            self.set_workspace(torch.empty(need, dtype=torch.uint8, device=f"cuda:{self.device}"))
+        return self._ws
+
+    def linear_transform(self, c0, c1, l: int, diag, g_baby: Sequence[int], k_baby: Sequence[KSK],
+                         g_giant: Sequence[int], k_giant: Sequence[KSK], out, stream=None):
+        """pc_linear_transform: diag [n2][n1][l][N] on the device; g_baby/k_baby the n1-1 baby
+        rotations, g_giant/k_giant the n2-1 giant rotations; out [2][l][N]."""
+        n2, n1 = int(diag.shape[0]), int(diag.shape[1])
+        assert len(g_baby) == len(k_baby) == n1 - 1 and len(g_giant) == len(k_giant) == n2 - 1
+        gb = (ctypes.c_uint32 * max(1, n1 - 1))(*g_baby)
+        kb = (_Ksk * max(1, n1 - 1))(*[k._c() for k in k_baby])
+        gg = (ctypes.c_uint32 * max(1, n2 - 1))(*g_giant)
+        kg = (_Ksk * max(1, n2 - 1))(*[k._c() for k in k_giant])
+        _ok(lib().pc_linear_transform(self._h, _ptr(c0), _ptr(c1), l, n1, gb, kb, n2, gg, kg, _ptr(diag), _ptr(out),
+                                      _stream(stream)), "pc_linear_transform")
+
     def expand_a(self, seed: bytes, l: int, out, stream=None):
         _ok(lib().pc_expand_a(self._h, bytes(seed), l, _ptr(out), _stream(stream)), "pc_expand_a")
 
     def check(self):
         _ok(lib().pc_check(self._h), "pc_check")
+
+    def set_checks(self, flags: int):
+        """pc_set_checks: 0, or CHECK_INPUTS to validate every input residue on the device."""
+        _ok(lib().pc_set_checks(self._h, flags), "pc_set_checks")
+
+    def last_error_word(self) -> int:
+        return int(lib().pc_last_error_word(self._h))
 
     def profile_begin(self, max_calls: int, every: int = 1):
         _ok(lib().pc_profile_begin(self._h, max_calls, every), "pc_profile_begin")

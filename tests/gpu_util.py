@@ -55,3 +55,17 @@ def random_key(P, seed=0):
     prim = [P.prime(g) for g in range(P.L + P.alpha)]
     b = np.stack([synth.uniform_residues(prim, P.N, seed, 0xB, j) for j in range(P.dnum)])
     return synth.chacha_seed(seed, 77), b
+
+
+def oracle_map(oracle, P, calls):
+    """Run independent oracle calls [(fn, args), ...] on the host's cores and
+    return their results in order.  The oracle's C entry points run without
+    the GIL (ctypes), so threads run them in parallel; the psi memo is filled
+    first so the threads only read it."""
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+    for g in range(P.L + P.alpha):
+        oracle.min_psi(P.prime(g), P.logN)
+    with ThreadPoolExecutor(max_workers=max(1, min(len(calls), os.cpu_count() or 1))) as ex:
+        futs = [ex.submit(fn, *args) for fn, args in calls]
+        return [f.result() for f in futs]

@@ -189,32 +189,6 @@ def test_rotation_n16_full_size(built, oracle):
     assert np.array_equal(G.host(o0), w0) and np.array_equal(G.host(o1), w1)
 
 
-def test_batch16_n16(built, oracle):
-    """16 ciphertexts under 16 rotation keys (2^k) in one batched call; each
-    checked against its own single-ciphertext GPU call, and three against the
-    oracle element by element."""
-    from key_switching_b200 import pc
-    P, C = G.contexts(oracle, 16, 24, 4, 31)
-    l, B = 24, 16
-    C.ensure_workspace(l, B)
-    keys, bs = [], []
-    for k in range(B):
-        seed, b = G.random_key(P, 100 + k)
-        bs.append(b)
-        keys.append(pc.KSK(seed, G.dev(b)))
-    ct = np.stack([np.stack([synth.uniform_residues(P.q, P.N, 7, k, h) for h in range(2)]) for k in range(B)])
-    out = G.empty(B, 2, l, P.N)
-    C.keyswitch_batch(G.dev(ct), B, l, keys, out)
-    got = G.host(out)
-    for k in [0, 7, 15]:
-        w0, w1 = oracle.keyswitch(P, ct[k, 0], ct[k, 1], l, keys[k].seed, bs[k])
-        assert np.array_equal(got[k, 0], w0) and np.array_equal(got[k, 1], w1), k
-    for k in range(B):
-        o0, o1 = G.empty(l, P.N), G.empty(l, P.N)
-        C.keyswitch(G.dev(ct[k, 0]), G.dev(ct[k, 1]), l, keys[k], o0, o1)
-        assert np.array_equal(got[k, 0], G.host(o0)) and np.array_equal(got[k, 1], G.host(o1)), k
-
-
 def test_batch_more_than_one_launch(built, oracle):
     """20 ciphertexts with 20 keys: the inner product runs in two launches of
     16 + 4 keys; every ciphertext bit-exact with the oracle (small ring)."""
@@ -272,3 +246,47 @@ def test_error_paths(built, oracle):
         C.ntt_fwd(c, 5, 2)  # primes beyond the basis
     assert ei.value.code == -1
     C.check()
+
+
+def test_input_checks_set_the_device_error_word(built, oracle):
+    """With PC_CHECK_INPUTS, a residue not below its prime in a ciphertext or
+    a key half sets the device error word (pc_check -> PC_E_DEVICE, word
+    bit PC_ERR_INPUT / PC_ERR_KEY); valid inputs leave it clear; without the
+    flag nothing is checked."""
+    from key_switching_b200 import pc
+    P, C = G.contexts(oracle, 12, 4, 2, 30)
+    l = 4
+    C.ensure_workspace(l)
+    seed, b = G.random_key(P, 61)
+    c0 = synth.uniform_residues(P.q[:l], P.N, 62, 0)
+    c1 = synth.uniform_residues(P.q[:l], P.N, 62, 1)
+    o0, o1 = G.empty(l, P.N), G.empty(l, P.N)
+    good = pc.KSK(seed, G.dev(b))
+    C.set_checks(pc.CHECK_INPUTS)
+    C.keyswitch(G.dev(c0), G.dev(c1), l, good, o0, o1)
+    C.check()                                   # valid inputs: word clear
+    w0, w1 = oracle.keyswitch(P, c0, c1, l, seed, b)
+    assert np.array_equal(G.host(o0), w0) and np.array_equal(G.host(o1), w1)
+    bad1 = c1.copy()
+    bad1[3, 1000] = 0xFFFFFFFF
+    C.keyswitch(G.dev(c0), G.dev(bad1), l, good, o0, o1)
+    with pytest.raises(pc.PCError) as ei:
+        C.check()
+    assert ei.value.code == -4 and C.last_error_word() == pc.ERR_INPUT
+    C.check()                                   # cleared by the previous check
+    bb = b.copy()
+    bb[1, P.L + 1, 7] = int(P.prime(P.L + 1))   # equal to its prime: not canonical
+    C.keyswitch(G.dev(c0), G.dev(c1), l, pc.KSK(seed, G.dev(bb)), o0, o1)
+    with pytest.raises(pc.PCError) as ei:
+        C.check()
+    assert ei.value.code == -4 and C.last_error_word() == pc.ERR_KEY
+    x = G.dev(np.stack([bad1] * 2))
+    C.ntt_fwd(x, 0, l, 2)
+    with pytest.raises(pc.PCError):
+        C.check()
+    C.set_checks(0)
+    C.keyswitch(G.dev(c0), G.dev(bad1), l, good, o0, o1)
+    C.check()                                   # not checked when off
+    with pytest.raises(pc.PCError) as ei:
+        C.set_checks(4)
+    assert ei.value.code == -1

@@ -174,31 +174,6 @@ def test_rotate_n16_full_size_real_key(built, oracle):
     assert _decrypt_rot_error(oracle, P, l, s, g, c0, c1, g0, g1) <= _bound(P, l, s, e)
 
 
-def test_rotate_hoisted_n16_full_size(built, oracle):
-    """N=2^16, l=24: four hoisted rotations (steps 1, 2, 4, 8) in one call;
-    two checked against the oracle element by element, the others against
-    single hoisted calls."""
-    from key_switching_b200 import pc
-    P, C = G.contexts(oracle, 16, 24, 4, 31)
-    l = 24
-    C.ensure_workspace(l, 4)
-    gs = [oracle.galois_elt(r, 16) for r in (1, 2, 4, 8)]
-    keys = [G.random_key(P, 300 + i) for i in range(4)]
-    kk = [pc.KSK(s, G.dev(b)) for s, b in keys]
-    c0, c1 = _ct(P, l, 6)
-    d0, d1 = G.dev(c0), G.dev(c1)
-    out = G.filled(4, 2, l, P.N)
-    C.rotate_hoisted(d0, d1, l, gs, kk, out)
-    got = G.host(out)
-    want = oracle.rotate_hoisted(P, c0, c1, l, [gs[0], gs[3]], [keys[0][0], keys[3][0]], [keys[0][1], keys[3][1]])
-    for i, (w0, w1) in zip([0, 3], want):
-        assert np.array_equal(got[i, 0], w0) and np.array_equal(got[i, 1], w1), i
-    for i in (1, 2):
-        one = G.filled(1, 2, l, P.N)
-        C.rotate_hoisted(d0, d1, l, [gs[i]], [kk[i]], one)
-        assert np.array_equal(G.host(one)[0], got[i]), i
-
-
 def test_relinearize_n12_real_key_decrypts(built, oracle):
     """The N=2^12, L=4, alpha=2 s^2 -> s key on a product of two ciphertexts:
     bit-exact, and c0' + c1' s matches d0 + d1 s + d2 s^2 within the bound."""

@@ -7,7 +7,12 @@ in a static device array of the library instead.  This test calls it through
 the C ABI and checks that its output equals pc_modup's bit for bit (the
 library's tolerance for integer results) on two calls in a row, that a size
 beyond its static scratch is refused, and that it needs no workspace.
-This file is collected last on purpose.
+
+The file is named so that pytest collects it last: the calls share one
+static array for the whole process, so these checks must hold after every
+other test has run in the same process (and they must also hold when the file
+runs alone in a fresh process); a run that stops at the first failure has
+then already run every other test.
 """
 import ctypes
 
@@ -27,7 +32,8 @@ def _noalloc(pc, ctx, c1, l, ext):
                                 ctypes.c_void_p(ext.data_ptr()), stream)
 
 
-@pytest.mark.parametrize("logN,L,alpha,bits,l", [(12, 4, 2, 30, 4), (16, 24, 4, 31, 24), (16, 24, 4, 31, 9)])
+@pytest.mark.parametrize("logN,L,alpha,bits,l", [(12, 4, 2, 30, 4), (16, 24, 4, 31, 24), (16, 24, 4, 31, 9),
+                                                   (16, 32, 4, 31, 32), (17, 16, 4, 31, 16)])
 def test_noalloc_matches_modup_twice(oracle, logN, L, alpha, bits, l):
     import torch
     from key_switching_b200 import build, pc
@@ -52,7 +58,7 @@ def test_noalloc_matches_modup_twice(oracle, logN, L, alpha, bits, l):
 def test_noalloc_rejects_sizes_beyond_its_scratch(oracle):
     from key_switching_b200 import pc
     P, C = G.contexts(oracle, 16, 34, 4, 31)
-    l = 33  # 33 * 2^16 words > 2^21
+    l = 33  # 33 * 2^16 words > 2^21 (32 * 2^16 = 2^21 is the largest accepted)
     c1 = G.empty(l, P.N)
     ext = G.empty(-(-l // 4), l + 4, P.N)
     assert _noalloc(pc, C, c1, l, ext) == -8
