@@ -24,6 +24,8 @@
 // call is canonical.
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+
 #include <cooperative_groups.h>
 
 #include <type_traits>
@@ -832,6 +834,191 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
     }
 }
 
+// ------------------------------------- inner product, warp-specialised
+// The fused inner product with regenerated 'a' (k_inner<FUSED, REGEN>'s
+// result) by two groups of NT = ROW_THREADS threads each.  Group 1 (the
+// producer) regenerates a_{j,g} with ChaCha12 for the CTA's rows, digit after
+// digit, into a double buffer in shared memory; it reads no data written by an
+// earlier kernel, so it starts while that kernel drains.  Group 0 (the
+// consumer) stages the column-pass tiles and the key's 'b' half one digit
+// ahead with asynchronous copies, runs the forward row passes and
+// multiply-accumulates both halves.  So the ALU-bound cipher and the
+// multiply-bound transforms run in different warps and overlap on the SM.
+// Hand-off: named barriers FULL[s] (ids 2, 3: the producer arrives once
+// digit j's words are in buffer s = j mod 2, the consumer waits) and
+// EMPTY[s] (ids 4, 5: the consumer arrives once it has read buffer s, if
+// digit j + 2 exists; the producer waits before refilling it); id 1 orders the
+// consumer group alone.  Every thread of a group takes the same barrier
+// steps (beta and the own digit are uniform over the CTA), so each barrier
+// phase completes.
+template <int LOGN>
+__global__ void __launch_bounds__(2 * Geo<LOGN>::ROW_THREADS, 2)
+k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
+           KeyPack kp, int pintt, u32 t0) {
+    using GE = Geo<LOGN>;
+    using PL = Plan<GE::LOGC>;
+    using PF = typename PL::P0;
+    using PLAST = typename LastPhase<GE::LOGC>::type;
+    static_assert(PLAST::KK == 16, "a thread's 16 coefficients are two whole ChaCha blocks");
+    constexpr int NT = GE::ROW_THREADS;
+    extern __shared__ __align__(16) u32 dyn[];
+    uint2 *stw = reinterpret_cast<uint2 *>(dyn);           // [NL][C] row twiddles
+    u32 *sm = dyn + 2 * GE::NL * GE::C;                      // [NL][ROW_LS] exchange
+    u32 *tiles = sm + GE::NL * GE::ROW_LS;                   // [2][C*8] column-pass tiles
+    uint4 *bbuf = reinterpret_cast<uint4 *>(tiles + 2 * GE::C * 8);  // [2][4][NT] key 'b' words
+    u32 *abuf = tiles + 2 * GE::C * 8 + 2 * 16 * NT;          // [2][16][NT] regenerated 'a'
+    __shared__ __align__(16) u32 spre[12 * MAX_L];
+    const bool producer = threadIdx.x >= NT;
+    const int tid = producer ? threadIdx.x - NT : threadIdx.x;
+    const int rho = tid / GE::TPR, lt = tid % GE::TPR;
+    const int row0 = blockIdx.x * GE::NL, row = row0 + rho;
+    const u32 t = t0 + blockIdx.y, z = blockIdx.z;
+    const u32 ll = l + T.alpha, beta = (l + T.alpha - 1) / T.alpha;
+    const u32 g = glob_of(T, l, t);
+    const PrimeK pk = T.pk[g];
+    const u32 q = pk.q;
+    const size_t rowoff = (size_t)row * GE::C;
+    const u32 jown = t < l ? t / T.alpha : beta;  // the digit holding t, if any
+    // set-up: the consumer stages this CTA's forward row twiddles; producer
+    // threads compute the counter-free quarter rounds of every digit's blocks
+    if (!producer) stage_row_tw<GE>(stw, T.rowF + (size_t)g * GE::N + (size_t)row0 * GE::C);
+    if (producer && (u32)tid < beta) {
+        u32 sd[8], pre[12];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sd[i] = kp.seed[z][i];
+        chacha12_precolumn(sd, g, tid, pre);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) spre[12 * tid + i] = pre[i];
+    }
+    __syncthreads();
+    if (producer) {
+        pdl_trigger();
+        u32 seed[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) seed[i] = kp.seed[z][i];
+        const u32 base = (u32)(rowoff + PLAST::x_of(lt, 0));
+        for (u32 j = 0; j < beta; ++j) {
+            const int s = j & 1;
+            if (j >= 2) bar_sync(4 + s, 2 * NT);
+            u32 o0[16], o1[16], pre[12];
+            const uint4 *pp = reinterpret_cast<const uint4 *>(spre + 12 * j);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const uint4 w4 = pp[i];
+                pre[4 * i] = w4.x; pre[4 * i + 1] = w4.y; pre[4 * i + 2] = w4.z; pre[4 * i + 3] = w4.w;
+            }
+            chacha12_block2_pre(pre, seed, base >> 3, g, j, o0, o1);
+            u32 *ab = abuf + s * 16 * NT + tid;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                // a * 2^-32 mod q from the 64-bit word pair
+                ab[w * NT] = redc(o0[2 * w], mod32(o0[2 * w + 1], q, pk.q1s), q, pk.qn);
+                ab[(8 + w) * NT] = redc(o1[2 * w], mod32(o1[2 * w + 1], q, pk.q1s), q, pk.qn);
+            }
+            bar_arrive(2 + s, 2 * NT);
+        }
+        return;
+    }
+    pdl_wait();
+    pdl_trigger();
+    const u32 *srcz_p = src + z * srcz;
+    const u32 *kb = kp.b[z] + (size_t)g * GE::N + rowoff + PLAST::x_of(lt, 0);
+    const size_t LLN = (size_t)(T.L + T.alpha) * GE::N;
+    u32 *line = sm + rho * GE::ROW_LS;
+    const TwRow tw{stw + rho * GE::C};
+    const u32 nconv = beta - (jown < beta ? 1u : 0u);
+    auto conv_digit = [&](u32 k) { return k < jown ? k : k + 1; };  // k-th converted digit
+    auto stage_b = [&](u32 j) {
+        const uint4 *gb = reinterpret_cast<const uint4 *>(kb + (size_t)j * LLN);
+        uint4 *sb = bbuf + (j & 1) * 4 * NT + tid;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cp_async16(sb + c * NT, gb + c);
+    };
+    if (nconv) stage_cm_rows<GE>(tiles, srcz_p + ((size_t)conv_digit(0) * ll + t) * GE::N, row0);
+    stage_b(0);
+    cp_async_commit();
+
+    u64 sb[16], sa[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) { sb[r] = 0; sa[r] = 0; }
+    u32 kc = 0;
+    for (u32 j = 0; j < beta; ++j) {
+        const bool own = j == jown;
+        // digit j's tile and b words have landed; the buffers refilled below
+        // are no longer read by any consumer thread
+        cp_async_wait_all();
+        bar_sync(1, NT);
+        if (j + 1 < beta) stage_b(j + 1);
+        if (!own && kc + 1 < nconv)
+            stage_cm_rows<GE>(tiles + ((kc + 1) & 1) * GE::C * 8,
+                              srcz_p + ((size_t)conv_digit(kc + 1) * ll + t) * GE::N, row0);
+        cp_async_commit();
+        u32 v[16], bv[16], av[16];
+        if (own) {
+            gload<PLAST>(v, c1 + z * c1z + (size_t)t * GE::N + rowoff, lt);
+        } else {
+            const u32 *tl = tiles + (kc & 1) * GE::C * 8;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) v[r] = tl[cm_addr(PF::x_of(lt, r), rho)];
+            line_fwd<GE::LOGC>(v, line, lt, RowAddr{}, tw, q, SyncWarp{});
+            ++kc;
+        }
+        const uint4 *bb = bbuf + (j & 1) * 4 * NT + tid;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 w4 = bb[c * NT];
+            bv[4 * c] = w4.x; bv[4 * c + 1] = w4.y; bv[4 * c + 2] = w4.z; bv[4 * c + 3] = w4.w;
+        }
+        bar_sync(2 + (j & 1), 2 * NT);  // digit j's 'a' words are in
+        const u32 *ab = abuf + (j & 1) * 16 * NT + tid;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) av[r] = ab[r * NT];
+        if (j + 2 < beta) bar_arrive(4 + (j & 1), 2 * NT);
+        // multiply-accumulate; fold the 64-bit sums every two digits
+        const bool fold = (j & 1) && (j + 1 < beta);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const u32 e = red1(v[r], q);
+            sb[r] += (u64)e * bv[r];
+            sa[r] += (u64)e * av[r];
+            if (fold) {
+                sb[r] = fold64(sb[r], q, pk.q1s);
+                sa[r] = fold64(sa[r], q, pk.q1s);
+            }
+        }
+    }
+    // canonical sums: REDC divides by 2^32; regenerated a carries another 2^-32
+    u32 ob[16], oa[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        ob[r] = shoup(redc64(sb[r], q, pk.qn, pk.q1s), pk.r32, pk.r32s, q);
+        oa[r] = shoup(redc64(sa[r], q, pk.qn, pk.q1s), pk.r64, pk.r64s, q);
+    }
+    u32 *d0 = acc + z * accz + (size_t)t * GE::N;
+    u32 *d1 = acc + z * accz + (size_t)(ll + t) * GE::N;
+    if (pintt && t >= l) {
+        cp_async_wait_all();
+        bar_sync(1, NT);  // every reader of the forward table and the tiles is done
+        stage_row_tw<GE>(stw, T.rowI + (size_t)g * GE::N + (size_t)row0 * GE::C);
+        cp_async_wait_all();
+        bar_sync(1, NT);
+        line_inv<GE::LOGC>(ob, line, lt, RowAddr{}, tw, q, SyncWarp{});
+        line_inv<GE::LOGC>(oa, line, lt, RowAddr{}, tw, q, SyncWarp{});
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int a = cm_addr(PF::x_of(lt, r), rho);
+            tiles[a] = ob[r];
+            tiles[GE::C * 8 + a] = oa[r];
+        }
+        bar_sync(1, NT);
+        store_cm_rows<GE>(tiles, d0, row0);
+        store_cm_rows<GE>(tiles + GE::C * 8, d1, row0);
+    } else {
+        gstore<PLAST>(ob, d0 + rowoff, lt);
+        gstore<PLAST>(oa, d1 + rowoff, lt);
+    }
+}
+
 // element z of a parameter array without copying the array to local memory
 __device__ __forceinline__ u32 pick(const u32 (&a)[KEYS_PER_LAUNCH], u32 z) {
     u32 v = a[0];
@@ -1033,10 +1220,26 @@ static size_t colconv_smem(const pc_ctx *c) {
     return sizeof(u32) * (size_t)2 * c->alpha * GE::CPW * GE::COL_LS;
 }
 
+// k_inner_ws: the key 'b' and regenerated 'a' double buffers of its two groups
+template <class GE>
+static constexpr size_t inner_ws_smem() {
+    return row_smem_bytes<GE>(2) + sizeof(u32) * 2 * 2 * 16 * GE::ROW_THREADS;
+}
+
 // k_inner with ROT: the packed source columns, 4 words per thread
 template <class GE>
 static constexpr size_t inner_rot_extra() {
     return sizeof(u32) * 4 * GE::ROW_THREADS;
+}
+
+// the warp-specialised inner product (PC_INNER_WS=0 at the first launch
+// selects the single-group kernel, for measurement)
+static bool use_inner_ws() {
+    static const bool on = [] {
+        const char *v = getenv("PC_INNER_WS");
+        return !(v && v[0] == '0');
+    }();
+    return on;
 }
 
 template <class F>
@@ -1055,6 +1258,8 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, false>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, false>, row_smem_bytes<GE>(2));
+        if constexpr (LastPhase<GE::LOGC>::type::KK == 16)
+            if (e == cudaSuccess) e = allow_smem(k_inner_ws<LG>, inner_ws_smem<GE>());
         if (e == cudaSuccess) e = allow_smem(k_inner_rot<LG, true>, row_smem_bytes<GE>(2) + inner_rot_extra<GE>());
         if (e == cudaSuccess) e = allow_smem(k_inner_rot<LG, false>, row_smem_bytes<GE>(2) + inner_rot_extra<GE>());
         if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_PLAIN>, row_smem_bytes<GE>(2));
@@ -1134,6 +1339,9 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
         dim3 grid(GE::ROW_BLOCKS, nt, Z);
         const size_t sm = row_smem_bytes<GE>(2) + (rot ? inner_rot_extra<GE>() : 0);
         const int pi = pintt ? 1 : 0;
+        // the two-group kernel needs a thread's 16 coefficients to be two
+        // whole ChaCha blocks (rows of 256 words: N >= 2^12)
+        constexpr bool ws_ok = LastPhase<GE::LOGC>::type::KK == 16;
         auto go = [&](auto kern) {
             return launch_ex(c, kern, grid, dim3(GE::ROW_THREADS), sm, s, c->tab, src, srcz, c1, c1z, acc, accz, l,
                              kp, pi, t0);
@@ -1143,7 +1351,11 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
                              kp, pi, t0, *rot);
         };
         if (rot) e = regen ? go_rot(k_inner_rot<LG, true>) : go_rot(k_inner_rot<LG, false>);
-        else if (fused) e = regen ? go(k_inner<LG, true, true>) : go(k_inner<LG, true, false>);
+        else if (fused && regen && use_inner_ws() && ws_ok) {
+            if constexpr (LastPhase<GE::LOGC>::type::KK == 16)
+                e = launch_ex(c, k_inner_ws<LG>, grid, dim3(2 * GE::ROW_THREADS), inner_ws_smem<GE>(), s, c->tab, src,
+                              srcz, c1, c1z, acc, accz, l, kp, pi, t0);
+        } else if (fused) e = regen ? go(k_inner<LG, true, true>) : go(k_inner<LG, true, false>);
         else e = regen ? go(k_inner<LG, false, true>) : go(k_inner<LG, false, false>);
     });
     return e;

@@ -187,6 +187,18 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
+// Named hardware barriers (ids 1..15; id 0 is __syncthreads): bar_sync
+// waits until `count` threads (a multiple of 32) have arrived at barrier id
+// in this phase, bar_arrive arrives without waiting.  Shared-memory writes made
+// before an arrive are visible to the threads that pass the matching sync.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+
 // Programmatic dependent launch: pdl_wait() blocks until the previous grid on
 // the stream has completed and its writes are visible (a no-op when the
 // kernel was launched without the attribute); pdl_trigger() lets the next
