@@ -125,6 +125,18 @@ def op_counts(wl, l: int, regen: bool = True):
         key_bytes = ks["bytes"] - 4 * l * N * 4
         return {"modmuls": up + n * (ks["modmuls"] - up), "bytes": 2 * l * N * 4 + n * (key_bytes + 2 * l * N * 4),
                 "chacha_blocks": n * ks["chacha_blocks"]}
+    if wl.op == "bsgs":
+        # n1 - 1 hoisted baby rotations (one ModUp), n2 - 1 giant rotations,
+        # n1 n2 diagonal products per half; bytes: ciphertext in and out, the
+        # keys' b halves, the diagonals
+        n1, n2 = wl.bsgs
+        st = stage_modmuls(wl.logN, wl.L, wl.alpha, l)
+        up = st["intt_row_c1"] + st["modup_col"]
+        baby = (up + (n1 - 1) * (ks["modmuls"] - up)) if n1 > 1 else 0
+        key_bytes = ks["bytes"] - 4 * l * N * 4
+        return {"modmuls": baby + (n2 - 1) * ks["modmuls"] + 2 * n1 * n2 * l * N,
+                "bytes": 4 * l * N * 4 + (n1 + n2 - 2) * key_bytes + n1 * n2 * l * N * 4,
+                "chacha_blocks": (n1 + n2 - 2) * ks["chacha_blocks"]}
     return ks
 
 
@@ -267,6 +279,10 @@ def workload_metric(wl) -> str:
     if wl.op in ("rotate", "hoisted"):
         return (f"rotations/s at N=2^{wl.logN} ({'single' if wl.op == 'rotate' else f'{wl.n_rot} hoisted'}"
                 " rotation(s) per ciphertext; 1 B200)")
+    if wl.op == "bsgs":
+        n1, n2 = wl.bsgs
+        return (f"baby-step giant-step linear transforms/s at N=2^{wl.logN}, levels {wl.levels[0]}..{wl.levels[-1]} "
+                f"({n2}x{n1} diagonals: {n1 - 1} hoisted baby and {n2 - 1} giant rotations each; 1 B200)")
     if wl.op == "relin":
         return f"ciphertext products (tensor + relinearisation) per second at N=2^{wl.logN} (1 B200)"
     if wl.logN == 16:
@@ -331,14 +347,18 @@ def run_ours(args):
         levels = list(wl.levels) if wl.levels else [L]
         B = len(items)  # this rank's ciphertexts per step
         nk = wl.n_rot if wl.op == "hoisted" else B  # keys per step
-        ctx.ensure_workspace(max(levels), max(B, min(wl.n_rot, 16)) if wl.op == "hoisted" else B)
+        if wl.op == "bsgs":
+            nk = wl.bsgs[0] + wl.bsgs[1] - 2
+            ctx.ensure_linear_transform_workspace(max(levels), wl.bsgs[0])
+        else:
+            ctx.ensure_workspace(max(levels), max(B, min(wl.n_rot, 16)) if wl.op == "hoisted" else B)
         per_set = (B * (2 * L * N * 4) * (2 if wl.op == "relin" else 1)
                    + nk * wl.dnum * (L + A) * N * 4 * (1 if regen else 2))
         nsets = max(2, math.ceil(2 * L2_BYTES / per_set)) if args.workload != "sweep_n17" else 1
         sets = []
         nct = B * (2 if wl.op == "relin" else 1)
         for s in range(nsets):
-            key_ids = items if wl.op != "hoisted" else range(nk)
+            key_ids = items if wl.op not in ("hoisted", "bsgs") else range(nk)
             keys = [make_key(1000 * s + k + 1) for k in key_ids]
             ct = dev(np.stack([np.stack([synth.uniform_residues(q, N, 50 + s, rank, k, h) for h in range(2)])
                                for k in (items if wl.op != "relin" else range(nct))]))
@@ -346,6 +366,20 @@ def run_ours(args):
         out = torch.empty((max(B, wl.n_rot), 2, L, N), dtype=torch.int32, device="cuda")
         units_per_step = (wl.n_rot if wl.op == "hoisted" else B) * len(levels)
         rot_gs = [pow(5, 1 << r, 2 * N) for r in range(wl.n_rot)]  # steps 1, 2, 4, ...
+        diags = {}
+        if wl.op == "bsgs":
+            # per level: [n2][n1][l][N] uniform plaintext diagonals, drawn on
+            # the device from a seeded generator (residue r of limb i mod q_i)
+            n1, n2 = wl.bsgs
+            gen = torch.Generator(device="cuda")
+            gen.manual_seed(1234 + rank)
+            qv = torch.tensor(q, dtype=torch.int64, device="cuda")
+            for l in levels:
+                r = torch.randint(0, 2**62, (n2, n1, l, N), generator=gen, device="cuda", dtype=torch.int64)
+                diags[l] = (r % qv[:l].view(1, 1, l, 1)).to(torch.int32).contiguous()
+            lt_gb = [pow(5, j, 2 * N) for j in range(1, n1)]           # baby rotations by 1 .. n1-1
+            lt_gg = [pow(5, n1 * i, 2 * N) for i in range(1, n2)]      # giant rotations by n1, 2 n1, ...
+            out_flat = out.view(-1)
 
         def run_op(ct, keys, st):
             """One step's library calls on stream st."""
@@ -356,6 +390,10 @@ def run_ours(args):
                     ctx.rotate_hoisted(ct[0, 0, :l], ct[0, 1, :l], l, rot_gs, keys, out[:, :, :l], st)
                 elif wl.op == "relin":
                     ctx.relinearize(ct[0, :, :l], ct[1, :, :l], l, keys[0], out[0, :, :l], st)
+                elif wl.op == "bsgs":
+                    n1 = wl.bsgs[0]
+                    ctx.linear_transform(ct[0, 0, :l], ct[0, 1, :l], l, diags[l], lt_gb, keys[:n1 - 1], lt_gg,
+                                         keys[n1 - 1:], out_flat[:2 * l * N].view(2, l, N), st)
                 elif B == 1:
                     # level-l ciphertext = the first l limbs of each half
                     ctx.keyswitch(ct[0, 0, :l], ct[0, 1, :l], l, keys[0], out[0, 0, :l], out[0, 1, :l], st)
@@ -379,6 +417,11 @@ def run_ours(args):
         if wl.op == "hoisted":  # one ModUp (2), then per batch of up to 16 rotations 4 (3 when serial)
             launches_per_step = (2 + (3 if os.environ.get("PC_NO_OVERLAP") else 4) * -(-wl.n_rot // 16)) \
                 * len(levels)
+        if wl.op == "bsgs":  # baby steps as hoisted rotations, one product kernel, a rotation per giant step
+            n1, n2 = wl.bsgs
+            fin = 3 if os.environ.get("PC_NO_OVERLAP") else 4
+            launches_per_step = ((2 + fin * -(-(n1 - 1) // 16) if n1 > 1 else 0) + 1
+                                 + (n2 - 1) * (2 + fin)) * len(levels)
         work = [op_counts(wl, l, regen) for l in levels]
 
     clocks = ClockSampler(local)
@@ -408,7 +451,7 @@ def run_ours(args):
     # the timed region (each runs its kernels serially on the stream, with an
     # event between consecutive kernels)
     stage_calls = []
-    if run_op is not None and wl.op != "hoisted":
+    if run_op is not None and wl.op not in ("hoisted", "bsgs"):
         n_prof = max(10, min(args.steps, 30)) if len(levels) == 1 else 10
         for k in range(n_prof):
             ctx.profile_begin(len(levels), 1)
@@ -545,14 +588,14 @@ def run_ours(args):
 # oracle's prime generator and imports nothing of the CUDA library.
 
 CPU_BASELINE_WORKLOADS = ("rot1_n16", "relin_n12", "ntt_n16", "rotate_n16", "relin_mul_n12", "relin_mul_n16",
-                          "hoisted8_n16", "batch16_n16", "sweep_n17")
+                          "hoisted8_n16", "batch16_n16", "sweep_n17", "bsgs_n17")
 
 
 def _unit(wl):
     if wl.name == "ntt_n16":
         return "limb-NTTs/s"
-    return {"rotate": "rotations/s", "hoisted": "rotations/s", "relin": "relinearisations/s"}.get(
-        wl.op, "key-switches/s")
+    return {"rotate": "rotations/s", "hoisted": "rotations/s", "relin": "relinearisations/s",
+            "bsgs": "linear-transforms/s"}.get(wl.op, "key-switches/s")
 
 
 class OracleJob:
@@ -576,6 +619,12 @@ class OracleJob:
             self.q = prim[0]
             return
         self.b = np.stack([synth.uniform_residues(prim, P.N, 1, 0xB, j) for j in range(P.dnum)])
+        if wl.op == "bsgs":
+            # a bounded sample of the level sweep: transforms at its mean level
+            self.l = sum(wl.levels) // len(wl.levels)
+            n1, n2 = wl.bsgs
+            self.diag = np.stack([np.stack([synth.uniform_residues(P.q[:self.l], P.N, 52, tag, i, j)
+                                            for j in range(n1)]) for i in range(n2)])
         self.c0 = synth.uniform_residues(P.q[:self.l], P.N, 50, tag, 0, 0)
         self.c1 = synth.uniform_residues(P.q[:self.l], P.N, 50, tag, 0, 1)
         self.y0 = synth.uniform_residues(P.q[:self.l], P.N, 51, tag, 0, 0)
@@ -597,6 +646,12 @@ class OracleJob:
             return wl.n_rot
         elif wl.op == "relin":
             O.relinearize(P, self.c0, self.c1, self.y0, self.y1, l, self.seed, self.b)
+        elif wl.op == "bsgs":
+            n1, n2 = wl.bsgs
+            gb = [pow(5, j, 2 * P.N) for j in range(1, n1)]
+            gg = [pow(5, n1 * i, 2 * P.N) for i in range(1, n2)]
+            O.linear_transform(P, self.c0, self.c1, l, self.diag, gb, [self.seed] * (n1 - 1), [self.b] * (n1 - 1),
+                               gg, [self.seed] * (n2 - 1), [self.b] * (n2 - 1))
         else:
             O.keyswitch(P, self.c0, self.c1, l, self.seed, self.b)
         return 1
@@ -732,7 +787,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="rot1_n16",
                     choices=["rot1_n16", "relin_n12", "batch16_n16", "ntt_n16", "sweep_n17", "rotate_n16",
-                             "hoisted8_n16", "relin_mul_n12", "relin_mul_n16"])
+                             "hoisted8_n16", "relin_mul_n12", "relin_mul_n16", "bsgs_n17"])
     ap.add_argument("--keys", default="regen", choices=["regen", "stored"])
     ap.add_argument("--no-graph", action="store_true",
                     help="call the library every step instead of replaying a CUDA graph of the step")

@@ -328,9 +328,12 @@ const char *pc_strerror(int code);
  * two variables; kind 2: ChaCha12 blocks; kind 3: 32-bit multiply-add; kind
  * 4: xor + add; kinds 5..8: ChaCha12 blocks with some rotations computed on
  * the multiply pipe; kind 9: ChaCha12, two interleaved blocks; kind 10:
- * ChaCha12 with the 16- and 8-bit rotations as byte permutes) over all SMs
- * and writes the operations per second to *ops_per_s (modmuls/s, or ChaCha
- * blocks/s).
+ * ChaCha12 with the 16- and 8-bit rotations as byte permutes; kinds 11..15:
+ * single instructions of the transforms and the cipher, to find the pipe each
+ * one issues on -- the conditional subtraction min(x, x - q), a funnel-shift
+ * rotation, a byte-permute rotation, a 64-bit addition, a compare-and-select
+ * subtraction) over all SMs and writes the operations per second to
+ * *ops_per_s (modmuls/s, ChaCha blocks/s, or instructions/s).
  * Synchronous.  Returns PC_OK, PC_E_ARG or PC_E_CUDA. */
 int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s);
 

@@ -50,9 +50,13 @@ namespace pc {
 #ifndef PC_INNER_MIN_CTAS
 #define PC_INNER_MIN_CTAS 4
 #endif
+#ifndef PC_MODDOWN_MIN_CTAS
+#define PC_MODDOWN_MIN_CTAS 6
+#endif
 constexpr int ROW_MIN_CTAS = PC_ROW_MIN_CTAS;
 constexpr int COLCONV_MIN_CTAS = PC_COLCONV_MIN_CTAS;
 constexpr int INNER_MIN_CTAS = PC_INNER_MIN_CTAS;
+constexpr int MODDOWN_MIN_CTAS = PC_MODDOWN_MIN_CTAS;
 
 // ------------------------------------------------------------------ helpers
 
@@ -1046,7 +1050,7 @@ k_inner_rot(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u3
 // half 0 of the giant-step operand of mac, read through X -> X^rp.galois[0],
 // added instead of c0, and both results added to out0 / out1 in place).
 template <int LOGN, int XF>
-__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
+__global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, MODDOWN_MIN_CTAS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, RotPack rp, const u32 *rx, const u32 *ry,
               MacIn mac) {
@@ -1073,11 +1077,18 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
     pdl_trigger();
     stage_cm_rows<GE>(tiles, U + z * Uz + (size_t)i * GE::N, row0);
     stage_cm_rows<GE>(tiles + GE::C * 8, U + z * Uz + ((size_t)l + i) * GE::N, row0);
+    // both halves' accumulator rows (and c0's row) load while the tiles stage
+    u32 ah[2][16], c0v[16];
+    gload<PLAST>(ah[0], acc + z * accz + (size_t)i * GE::N + rowoff, lt);
+    gload<PLAST>(ah[1], acc + z * accz + ((size_t)ll + i) * GE::N + rowoff, lt);
+    if constexpr (XF == XF_PLAIN) {
+        if (c0) gload<PLAST>(c0v, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
+    }
     cp_async_wait_all();
     __syncthreads();
     auto half = [&](const int h) {
-        u32 v[16], a[16];
-        gload<PLAST>(a, acc + z * accz + ((size_t)h * ll + i) * GE::N + rowoff, lt);
+        u32 v[16];
+        const u32 *a = ah[h];
         const u32 *tl = tiles + h * GE::C * 8;
 #pragma unroll
         for (int r = 0; r < 16; ++r) v[r] = tl[cm_addr(PF::x_of(lt, r), rho)];
@@ -1122,7 +1133,8 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
                 load_row_in<PLAST, LOGN, GE::C>(cc, c0 + z * c0z + (size_t)i * GE::N, nullptr, row, lt,
                                                 pick(rp.galois, z), pk);
             else
-                gload<PLAST>(cc, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) cc[r] = c0v[r];
 #pragma unroll
             for (int r = 0; r < 16; ++r) o[r] = red1(o[r] + cc[r], q);
         }
@@ -1247,6 +1259,13 @@ static cudaError_t allow_smem(F *f, size_t bytes) {
     return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+template <int LG>
+static cudaError_t allow_inner_ws() {
+    using GE = Geo<LG>;
+    if constexpr (LastPhase<GE::LOGC>::type::KK == 16) return allow_smem(k_inner_ws<LG>, inner_ws_smem<GE>());
+    else return cudaSuccess;
+}
+
 cudaError_t prepare_kernels(const pc_ctx *c) {
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
@@ -1258,8 +1277,7 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, false, false>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, true>, row_smem_bytes<GE>(2));
         if (e == cudaSuccess) e = allow_smem(k_inner<LG, true, false>, row_smem_bytes<GE>(2));
-        if constexpr (LastPhase<GE::LOGC>::type::KK == 16)
-            if (e == cudaSuccess) e = allow_smem(k_inner_ws<LG>, inner_ws_smem<GE>());
+        if (e == cudaSuccess) e = allow_inner_ws<LG>();
         if (e == cudaSuccess) e = allow_smem(k_inner_rot<LG, true>, row_smem_bytes<GE>(2) + inner_rot_extra<GE>());
         if (e == cudaSuccess) e = allow_smem(k_inner_rot<LG, false>, row_smem_bytes<GE>(2) + inner_rot_extra<GE>());
         if (e == cudaSuccess) e = allow_smem(k_moddown_row<LG, XF_PLAIN>, row_smem_bytes<GE>(2));
@@ -1328,6 +1346,20 @@ cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t src
     return e;
 }
 
+// the two-group inner product where a thread's 16 coefficients are two whole
+// ChaCha blocks (rows of 256 words, N >= 2^12); instantiated only there
+template <int LG>
+static cudaError_t launch_inner_ws(const pc_ctx *c, dim3 grid, cudaStream_t s, const u32 *src, size_t srcz,
+                                   const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l, const KeyPack &kp,
+                                   int pi, u32 t0) {
+    using GE = Geo<LG>;
+    if constexpr (LastPhase<GE::LOGC>::type::KK == 16)
+        return launch_ex(c, k_inner_ws<LG>, grid, dim3(2 * GE::ROW_THREADS), inner_ws_smem<GE>(), s, c->tab, src,
+                         srcz, c1, c1z, acc, accz, l, kp, pi, t0);
+    else
+        return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t srcz, const u32 *c1, size_t c1z,
                          u32 *acc, size_t accz, u32 l, const KeyPack &kp, u32 Z, bool regen, bool pintt,
                          cudaStream_t s, u32 t0, u32 nt, const RotPack *rot) {
@@ -1351,11 +1383,9 @@ cudaError_t launch_inner(const pc_ctx *c, bool fused, const u32 *src, size_t src
                              kp, pi, t0, *rot);
         };
         if (rot) e = regen ? go_rot(k_inner_rot<LG, true>) : go_rot(k_inner_rot<LG, false>);
-        else if (fused && regen && use_inner_ws() && ws_ok) {
-            if constexpr (LastPhase<GE::LOGC>::type::KK == 16)
-                e = launch_ex(c, k_inner_ws<LG>, grid, dim3(2 * GE::ROW_THREADS), inner_ws_smem<GE>(), s, c->tab, src,
-                              srcz, c1, c1z, acc, accz, l, kp, pi, t0);
-        } else if (fused) e = regen ? go(k_inner<LG, true, true>) : go(k_inner<LG, true, false>);
+        else if (fused && regen && use_inner_ws() && ws_ok)
+            e = launch_inner_ws<LG>(c, grid, s, src, srcz, c1, c1z, acc, accz, l, kp, pi, t0);
+        else if (fused) e = regen ? go(k_inner<LG, true, true>) : go(k_inner<LG, true, false>);
         else e = regen ? go(k_inner<LG, false, true>) : go(k_inner<LG, false, false>);
     });
     return e;

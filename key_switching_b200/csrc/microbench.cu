@@ -14,6 +14,11 @@
 //         (mask 1: rot16; 5: rot16+rot8; 3: rot16+rot12; 15: all) -> blocks/s
 //   9: ChaCha12, two blocks with interleaved quarter rounds  -> blocks/s
 //  10: ChaCha12 with the 16- and 8-bit rotations as byte permutes -> blocks/s
+//  11: conditional subtraction min(x, x - q) (the lazy reduction) -> ops/s
+//  12: 32-bit rotation by a funnel shift                    -> ops/s
+//  13: 32-bit rotation by a byte permute                    -> ops/s
+//  14: 64-bit addition                                      -> ops/s
+//  15: conditional subtraction by compare and select        -> ops/s
 #include <cuda_runtime.h>
 
 #include "chacha.cuh"
@@ -86,6 +91,29 @@ __global__ void __launch_bounds__(MB_THREADS) k_micro(u32 iters, u32 q, u32 w, u
 #pragma unroll
             for (int i = 0; i < 4; ++i) m[i] = mul[i] ^ (ws & 0x80000000u & qn);  // opaque to the compiler
             micro_chacha<MASK>(x, it, tid, m);
+        } else if constexpr (KIND == 11) {
+#pragma unroll
+            for (int i = 0; i < MB_CHAINS; ++i) x[i] = red1(x[i] + w, q);
+        } else if constexpr (KIND == 12) {
+#pragma unroll
+            for (int i = 0; i < MB_CHAINS; ++i) x[i] = __funnelshift_l(x[i], x[i], 7);
+        } else if constexpr (KIND == 13) {
+#pragma unroll
+            for (int i = 0; i < MB_CHAINS; ++i) x[i] = __byte_perm(x[i], x[i], 0x2103);
+        } else if constexpr (KIND == 14) {
+#pragma unroll
+            for (int i = 0; i < MB_CHAINS / 2; ++i) {
+                u64 a = ((u64)x[2 * i] << 32) | x[2 * i + 1];
+                a += ((u64)y[i] << 32) | w;
+                x[2 * i] = (u32)(a >> 32);
+                x[2 * i + 1] = (u32)a;
+            }
+        } else if constexpr (KIND == 15) {
+#pragma unroll
+            for (int i = 0; i < MB_CHAINS; ++i) {
+                const u32 t = x[i] + w;
+                x[i] = t >= q ? t - q : t;
+            }
         } else if constexpr (KIND == 3) {
 #pragma unroll
             for (int i = 0; i < MB_CHAINS; ++i) x[i] = x[i] * y[i] + w;
@@ -126,7 +154,7 @@ static cudaError_t run_micro(int sms, u32 iters, u32 *sink, float *ms) {
 
 extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s) {
     using namespace pc;
-    if (!ops_per_s || kind < 0 || kind > 10 || iters < 1) return PC_E_ARG;
+    if (!ops_per_s || kind < 0 || kind > 15 || iters < 1) return PC_E_ARG;
     if (cudaSetDevice(device) != cudaSuccess) return PC_E_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return PC_E_CUDA;
@@ -145,6 +173,11 @@ extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_p
         case 8: e = run_micro<8>(sms, iters, sink, &ms); break;
         case 9: e = run_micro<9>(sms, iters, sink, &ms); break;
         case 10: e = run_micro<10>(sms, iters, sink, &ms); break;
+        case 11: e = run_micro<11>(sms, iters, sink, &ms); break;
+        case 12: e = run_micro<12>(sms, iters, sink, &ms); break;
+        case 13: e = run_micro<13>(sms, iters, sink, &ms); break;
+        case 14: e = run_micro<14>(sms, iters, sink, &ms); break;
+        case 15: e = run_micro<15>(sms, iters, sink, &ms); break;
         default: e = run_micro<4>(sms, iters, sink, &ms); break;
     }
     cudaFree(sink);

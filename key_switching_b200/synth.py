@@ -30,8 +30,9 @@ class Workload:
     key: str             # "square" (s^2 -> s) or "rot" (rotation keys)
     n_ct: int = 1        # ciphertexts per step
     levels: tuple = ()   # () = top level only
-    op: str = "keyswitch"  # "keyswitch", "rotate", "hoisted" (n_rot rotations, one ModUp), "relin"
+    op: str = "keyswitch"  # "keyswitch", "rotate", "hoisted" (n_rot rotations, one ModUp), "relin", "bsgs"
     n_rot: int = 1
+    bsgs: tuple = ()     # (n1, n2): baby and giant steps of a linear transform
 
     @property
     def N(self) -> int:
@@ -61,6 +62,10 @@ WORKLOADS = {
     # ciphertext product: tensor, then relinearisation with the s^2 -> s key
     "relin_mul_n12": Workload("relin_mul_n12", 12, 4, 2, 30, "ternary", "square", op="relin"),
     "relin_mul_n16": Workload("relin_mul_n16", 16, 24, 4, 31, "hw", "square", op="relin"),
+    # baby-step giant-step linear transform (4 x 4 diagonals: 3 hoisted baby
+    # rotations, 3 giant rotations) at every level of the N=2^17 sweep
+    "bsgs_n17": Workload("bsgs_n17", 17, 40, 5, 31, "hw", "rot", levels=tuple(range(40, 0, -1)), op="bsgs",
+                         bsgs=(4, 4)),
 }
 
 
