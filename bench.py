@@ -269,6 +269,15 @@ def launch_ranks(argv, n: int) -> int:
     return subprocess.call(cmd)
 
 
+def hbm_peak():
+    """(GB/s, source): the measured copy bandwidth of MEASURED_PEAKS.json when
+    the file is there, else the profiling recipe's fallback figure."""
+    try:
+        return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback 6650 GB/s (no measured-peaks file on this machine)"
+
+
 def workload_metric(wl) -> str:
     """The metric line of a workload (the N=2^16 key switch carries the
     headline metric's exact wording)."""
@@ -474,6 +483,30 @@ def run_ours(args):
                       "launch": "CUDA graph replay of every step" if graphs is not None else "library calls"},
            "gpu_launches": launches_per_step * args.steps, "clocks": clk}
 
+    if args.workload == "ntt_n16":
+        # forward + inverse NTT of 64 x 28 limbs: N/2 log N butterflies (one
+        # modular multiply each) per limb and direction, plus the inverse's
+        # N^-1 scale; bytes: every word read and written once per direction
+        NPL = L + A
+        mm = 2 * wl.n_ct * NPL * (N // 2 * wl.logN) + wl.n_ct * NPL * N
+        by = 2 * 2 * wl.n_ct * NPL * N * 4
+        sec_per_step = ms * 1e-3 / args.steps
+        peak_derived = SMS * IMAD_PER_SM_CLK * 1965e6 / MODMUL_IMAD
+        hbm, hbm_src = hbm_peak()
+        t_roof = max(by / (hbm * 1e9), mm / peak_derived)
+        res["step_roofline"] = {"modmuls_per_step": mm, "hbm_bytes_per_step": by,
+                                "achieved_gbs": by / sec_per_step / 1e9,
+                                "achieved_tmodmul_s": mm / sec_per_step / 1e12,
+                                "t_roofline_us": t_roof * 1e6, "t_step_us": sec_per_step * 1e6,
+                                "frac": t_roof / sec_per_step, "modmul_peak_derived": peak_derived,
+                                "hbm_peak_gbs": hbm, "hbm_peak_source": hbm_src}
+        peak_ops = SMS * ISSUE_LANES_PER_SM_CLK * 1965e6
+        res["roofline"] = {"bound": "alu", "kernel": "whole step (column and row passes)",
+                           "achieved": MODMUL_IMAD * mm / sec_per_step / 1e12, "peak": peak_ops / 1e12,
+                           "unit": "Tintop/s", "frac": MODMUL_IMAD * mm / sec_per_step / peak_ops, "traffic": None,
+                           "peak_source": "derived: 148 SMs x 128 issued 32-bit lane ops/clk x 1965 MHz; "
+                                          "ops = 4 per Shoup modular multiply"}
+
     if work is not None:
         nct = B  # this rank's ciphertexts per step
         mm = sum(w["modmuls"] for w in work)
@@ -484,11 +517,7 @@ def run_ours(args):
             peak_meas = pc.microbench(0, 2048, local) if rank == 0 else None
         except Exception:
             peak_meas = None
-        hbm_src = "MEASURED_PEAKS.json"
-        try:
-            hbm = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
-        except (OSError, KeyError, ValueError):
-            hbm, hbm_src = 6650.0, "fallback 6650 GB/s (MEASURED_PEAKS.json absent)"
+        hbm, hbm_src = hbm_peak()
         t_roof = max(by / (hbm * 1e9), mm / peak_derived)
         res["step_roofline"] = {"modmuls_per_step": mm * nct, "hbm_bytes_per_step": by * nct,
                                 "achieved_gbs": by * nct / sec_per_step / 1e9,

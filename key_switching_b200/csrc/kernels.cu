@@ -50,6 +50,9 @@ namespace pc {
 #ifndef PC_INNER_MIN_CTAS
 #define PC_INNER_MIN_CTAS 4
 #endif
+#ifndef PC_INNER_WS_MIN_CTAS
+#define PC_INNER_WS_MIN_CTAS 2
+#endif
 #ifndef PC_MODDOWN_MIN_CTAS
 #define PC_MODDOWN_MIN_CTAS 6
 #endif
@@ -856,7 +859,7 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
 // steps (beta and the own digit are uniform over the CTA), so each barrier
 // phase completes.
 template <int LOGN>
-__global__ void __launch_bounds__(2 * Geo<LOGN>::ROW_THREADS, 2)
+__global__ void __launch_bounds__(2 * Geo<LOGN>::ROW_THREADS, PC_INNER_WS_MIN_CTAS)
 k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
            KeyPack kp, int pintt, u32 t0) {
     using GE = Geo<LOGN>;

@@ -84,13 +84,6 @@ __global__ void __launch_bounds__(MB_THREADS) k_micro(u32 iters, u32 q, u32 w, u
             chacha12_block2(k, 2 * it, tid, 0, o0, o1);
 #pragma unroll
             for (int i = 0; i < 8; ++i) x[i] ^= o0[i] + o1[i + 8];
-        } else if constexpr (KIND >= 5) {
-            constexpr int MASK = KIND == 5 ? 1 : KIND == 6 ? 5 : KIND == 7 ? 3 : 15;
-            const u32 mul[4] = {w & 0 | (1u << 16), 1u << 12, 1u << 8, 1u << 7};
-            u32 m[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) m[i] = mul[i] ^ (ws & 0x80000000u & qn);  // opaque to the compiler
-            micro_chacha<MASK>(x, it, tid, m);
         } else if constexpr (KIND == 11) {
 #pragma unroll
             for (int i = 0; i < MB_CHAINS; ++i) x[i] = red1(x[i] + w, q);
@@ -114,6 +107,13 @@ __global__ void __launch_bounds__(MB_THREADS) k_micro(u32 iters, u32 q, u32 w, u
                 const u32 t = x[i] + w;
                 x[i] = t >= q ? t - q : t;
             }
+        } else if constexpr (KIND >= 5) {
+            constexpr int MASK = KIND == 5 ? 1 : KIND == 6 ? 5 : KIND == 7 ? 3 : 15;
+            const u32 mul[4] = {w & 0 | (1u << 16), 1u << 12, 1u << 8, 1u << 7};
+            u32 m[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m[i] = mul[i] ^ (ws & 0x80000000u & qn);  // opaque to the compiler
+            micro_chacha<MASK>(x, it, tid, m);
         } else if constexpr (KIND == 3) {
 #pragma unroll
             for (int i = 0; i < MB_CHAINS; ++i) x[i] = x[i] * y[i] + w;
@@ -183,7 +183,7 @@ extern "C" int pc_microbench(int device, int kind, uint32_t iters, double *ops_p
     cudaFree(sink);
     if (e != cudaSuccess || ms <= 0.f) return PC_E_CUDA;
     const double threads = (double)sms * 8 * MB_THREADS;
-    const double per_iter = kind == 9 ? 2.0 : (kind == 2 || kind >= 5) ? 1.0 : (double)MB_CHAINS;
+    const double per_iter = kind == 9 ? 2.0 : (kind == 2 || (kind >= 5 && kind <= 10)) ? 1.0 : (double)MB_CHAINS;
     *ops_per_s = threads * per_iter * (double)iters / (ms * 1e-3);
     return PC_OK;
 }

@@ -186,3 +186,24 @@ def test_standalone_calls_full_size(built, oracle, shape, l):
     C.moddown(G.dev(accr), l, out)
     assert np.array_equal(G.host(out), want_md)
     C.check()
+
+
+def test_hoisted_identity_equals_keyswitch_n16(n16, oracle):
+    """A hoisted rotation by g = 1 (k_inner_rot's body) equals the plain key
+    switch (the two-group inner product) bit for bit at N=2^16, l=24 and
+    l=9, both with a regenerated and with a stored 'a' half: the two inner
+    product texts are pinned against each other."""
+    from key_switching_b200 import pc
+    P, C = n16
+    for l, stored in ((24, False), (9, False), (24, True)):
+        C.ensure_workspace(l)
+        seed, b = G.random_key(P, 61 + l)
+        key = pc.KSK(seed, G.dev(b), G.dev(_stored_a(P, 61)) if stored else None)
+        c0, c1 = _ct(P, l, 62, l)
+        d0, d1 = G.dev(c0), G.dev(c1)
+        o0, o1 = G.filled(l, P.N), G.filled(l, P.N)
+        C.keyswitch(d0, d1, l, key, o0, o1)
+        h = G.filled(1, 2, l, P.N)
+        C.rotate_hoisted(d0, d1, l, [1], [key], h)
+        got = G.host(h)
+        assert np.array_equal(got[0, 0], G.host(o0)) and np.array_equal(got[0, 1], G.host(o1)), (l, stored)
