@@ -346,6 +346,12 @@ k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
 }
 
 // ------------------------------------------------- column conversion kernel
+// y tiles of the conversion kernel: each lane's 16 values of a source limb are
+// stored as one run of YT_LS words (16 + 4 padding), so the targets read them
+// with four 16-byte loads; lanes 20 words apart put any 8 consecutive lanes'
+// 16-byte accesses on distinct bank groups.
+constexpr int YT_LS = 20;
+
 // One CTA of alpha warps per (unit, strip of CPW columns); a column is held
 // by TPCOL consecutive lanes, so every exchange is warp-synchronous.
 //   mode 0 (ModUp):   unit = digit j; warp k < d runs the inverse column pass
@@ -394,20 +400,28 @@ __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *
 #pragma unroll
         for (int k = 0; k < D; ++k) cv0[k] = __ldg(conv0 + k);
         u32 v0[16];
+        // the lane's 16 values of source k are one contiguous run (see YT_LS)
+        const u32 *yl = sy + (c * GE::TPCOL + lt) * YT_LS;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int x = PF::x_of(lt, r);
-            const int xa = c * GE::COL_LS + x + (x >> 4);
-            u64 a0 = 0;
+        for (int rc = 0; rc < 4; ++rc) {
+            u64 a0[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int k = 0; k < D; ++k) {
-                if (k == 4 || k == 6) a0 = fold64(a0, q0, q1s0);
-                a0 += (u64)sy[k * GE::CPW * GE::COL_LS + xa] * cv0[k];
+                const uint4 y4 = *reinterpret_cast<const uint4 *>(yl + k * GE::CPW * GE::TPCOL * YT_LS + 4 * rc);
+                const u32 yv[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (k == 4 || k == 6) a0[i] = fold64(a0[i], q0, q1s0);
+                    a0[i] += (u64)yv[i] * cv0[k];
+                }
             }
-            if constexpr (D <= 4) v0[r] = redc((u32)a0, red1((u32)(a0 >> 32), q0), q0, qn0);
-            else v0[r] = redc64(a0, q0, qn0, q1s0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if constexpr (D <= 4) v0[4 * rc + i] = redc((u32)a0[i], red1((u32)(a0[i] >> 32), q0), q0, qn0);
+                else v0[4 * rc + i] = redc64(a0[i], q0, qn0, q1s0);
+            }
         }
-        line_fwd<GE::LOGR>(v0, xl0, lt, RowAddr{}, TwRowG{T.colF + (size_t)g0 * GE::R}, q0, SyncWarp{});
+        line_fwd<GE::LOGR>(v0, xl0, lt, Pad4Addr{}, TwRowG{T.colF + (size_t)g0 * GE::R}, q0, SyncWarp{});
         if constexpr (OUT_CM) {
             gstore<PLAST>(v0, dst0 + (size_t)col * GE::R, lt);
         } else {
@@ -428,9 +442,9 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int c = lane / GE::TPCOL, lt = lane % GE::TPCOL;
     const int col = blockIdx.x * GE::CPW + c;
-    u32 *sy = dyn;                                          // [alpha][CPW][COL_LS] y tiles
-    // one exchange line per warp and column
-    u32 *xl = dyn + (T.alpha + warp) * GE::CPW * GE::COL_LS + c * GE::COL_LS;
+    u32 *sy = dyn;                                          // [alpha][CPW][TPCOL][YT_LS] y tiles
+    // one exchange line per warp and column, after the y tiles
+    u32 *xl = dyn + T.alpha * GE::CPW * GE::TPCOL * YT_LS + (warp * GE::CPW + c) * GE::COL_LS4;
     const u32 units = mode == 0 ? (l + T.alpha - 1) / T.alpha : 2;
     const u32 z = blockIdx.z / units, unit = blockIdx.z % units;
     const u32 ll = l + T.alpha;
@@ -453,14 +467,14 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
         const u32 q = T.pk[gsrc].q;
         u32 v[16];
         gload<PLAST>(v, s0 + (size_t)warp * GE::N + (size_t)col * GE::R, lt);
-        line_inv<GE::LOGR>(v, xl, lt, RowAddr{}, TwRowG{T.colI + (size_t)gsrc * GE::R}, q, SyncWarp{});
+        line_inv<GE::LOGR>(v, xl, lt, Pad4Addr{}, TwRowG{T.colI + (size_t)gsrc * GE::R}, q, SyncWarp{});
         const uint2 sc = mode == 0 ? T.upScale[(size_t)(d - 1) * T.L + gsrc] : T.downScale[warp];
-        u32 *yt = sy + (warp * GE::CPW + c) * GE::COL_LS;
+        // the lane's 16 values (PF positions lt + TPCOL r) as one contiguous run
+        u32 *yt = sy + ((warp * GE::CPW + c) * GE::TPCOL + lt) * YT_LS;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int x = PF::x_of(lt, r);
-            yt[x + (x >> 4)] = shoup(v[r], sc.x, sc.y, q);
-        }
+        for (int r = 0; r < 16; r += 4)
+            *reinterpret_cast<uint4 *>(yt + r) = make_uint4(shoup(v[r], sc.x, sc.y, q), shoup(v[r + 1], sc.x, sc.y, q),
+                                                            shoup(v[r + 2], sc.x, sc.y, q), shoup(v[r + 3], sc.x, sc.y, q));
     }
     __syncthreads();
     switch (d) {  // uniform over the CTA
@@ -1232,7 +1246,7 @@ namespace PC_NS {
 // shared memory of k_colconv: alpha y tiles and one exchange line per warp
 template <class GE>
 static size_t colconv_smem(const pc_ctx *c) {
-    return sizeof(u32) * (size_t)2 * c->alpha * GE::CPW * GE::COL_LS;
+    return sizeof(u32) * ((size_t)c->alpha * GE::CPW * GE::TPCOL * YT_LS + (size_t)c->alpha * GE::CPW * GE::COL_LS4);
 }
 
 // k_inner_ws: the key 'b' and regenerated 'a' double buffers of its two groups

@@ -20,6 +20,8 @@
 // radix-16 phase) on them; phases exchange through shared memory.  A line
 // of M elements is handled by M/16 threads.
 #pragma once
+#include <type_traits>
+
 #include "modarith.cuh"
 
 namespace pc {
@@ -113,16 +115,47 @@ struct SyncCta {
     __device__ __forceinline__ void operator()() const { __syncthreads(); }
 };
 
+// Line layout with 16-byte exchanges: element x at x + 4 (x >> 4).  A lane's
+// run of 16 consecutive elements (a distance-1 phase) is then four aligned
+// 16-byte chunks, and with runs 20 words apart any 8 consecutive lanes' chunks
+// fall on distinct bank groups; a strided phase (elements lt + 16 r) touches
+// one word per lane, consecutive lanes on consecutive banks.  Lines need
+// M + M/4 words.
+struct Pad4Addr {
+    __device__ __forceinline__ int operator()(int x) const { return x + 4 * (x >> 4); }
+};
+
+template <class PH>
+struct IsRun16 {  // a thread holds 16 consecutive elements of the line
+    static constexpr bool value = PH::D == 1 && PH::KK == 16;
+};
+
 // Exchange the registers of phase A's layout into phase B's layout through
 // shared memory.  ADDR(x) gives the word address of element x of the line.
 template <class PA, class PB, class SYNC, class ADDR>
 __device__ __forceinline__ void exchange(u32 v[16], u32 *sm, int lt, const ADDR &addr, const SYNC &sync) {
+    constexpr bool pad4 = std::is_same<ADDR, Pad4Addr>::value;
     sync();
+    if constexpr (pad4 && IsRun16<PA>::value) {
+        uint4 *d = reinterpret_cast<uint4 *>(sm + addr(PA::x_of(lt, 0)));
 #pragma unroll
-    for (int r = 0; r < 16; ++r) sm[addr(PA::x_of(lt, r))] = v[r];
+        for (int c = 0; c < 4; ++c) d[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    } else {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sm[addr(PA::x_of(lt, r))] = v[r];
+    }
     sync();
+    if constexpr (pad4 && IsRun16<PB>::value) {
+        const uint4 *d = reinterpret_cast<const uint4 *>(sm + addr(PB::x_of(lt, 0)));
 #pragma unroll
-    for (int r = 0; r < 16; ++r) v[r] = sm[addr(PB::x_of(lt, r))];
+        for (int c = 0; c < 4; ++c) {
+            const uint4 w = d[c];
+            v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) v[r] = sm[addr(PB::x_of(lt, r))];
+    }
 }
 
 // Full forward line transform: registers enter at Plan::fwd_in positions and
@@ -234,6 +267,7 @@ struct Geo {
     // per TPCOL consecutive lanes, CPW columns per warp, warp barriers only
     static constexpr int CPW = 32 / TPCOL;
     static constexpr int COL_LS = R + R / 16;  // padded column stride in shared memory
+    static constexpr int COL_LS4 = R + R / 4;  // column stride of a Pad4Addr line
     static_assert(LOGC >= 4 && LOGR >= 4 && LOGR <= 9, "supported 2^8..2^17 (R,C >= 16)");
 };
 
