@@ -888,7 +888,7 @@ k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32
     u32 *tiles = sm + GE::NL * GE::ROW_LS;                   // [2][C*8] column-pass tiles
     uint4 *bbuf = reinterpret_cast<uint4 *>(tiles + 2 * GE::C * 8);  // [2][4][NT] key 'b' words
     u32 *abuf = tiles + 2 * GE::C * 8 + 2 * 16 * NT;          // [2][16][NT] regenerated 'a'
-    __shared__ __align__(16) u32 spre[12 * MAX_L];
+    u32 *spre = abuf + 2 * 16 * NT;                            // [beta][12] first-round words
     const bool producer = threadIdx.x >= NT;
     const int tid = producer ? threadIdx.x - NT : threadIdx.x;
     const int rho = tid / GE::TPR, lt = tid % GE::TPR;
@@ -1249,10 +1249,11 @@ static size_t colconv_smem(const pc_ctx *c) {
     return sizeof(u32) * ((size_t)c->alpha * GE::CPW * GE::TPCOL * YT_LS + (size_t)c->alpha * GE::CPW * GE::COL_LS4);
 }
 
-// k_inner_ws: the key 'b' and regenerated 'a' double buffers of its two groups
+// k_inner_ws: the key 'b' and regenerated 'a' double buffers of its two
+// groups, and the counter-free first-round words of each of the beta digits
 template <class GE>
-static constexpr size_t inner_ws_smem() {
-    return row_smem_bytes<GE>(2) + sizeof(u32) * 2 * 2 * 16 * GE::ROW_THREADS;
+static constexpr size_t inner_ws_smem(u32 beta) {
+    return row_smem_bytes<GE>(2) + sizeof(u32) * (2 * 2 * 16 * GE::ROW_THREADS + 12 * (size_t)beta);
 }
 
 // k_inner with ROT: the packed source columns, 4 words per thread
@@ -1279,7 +1280,7 @@ static cudaError_t allow_smem(F *f, size_t bytes) {
 template <int LG>
 static cudaError_t allow_inner_ws() {
     using GE = Geo<LG>;
-    if constexpr (LastPhase<GE::LOGC>::type::KK == 16) return allow_smem(k_inner_ws<LG>, inner_ws_smem<GE>());
+    if constexpr (LastPhase<GE::LOGC>::type::KK == 16) return allow_smem(k_inner_ws<LG>, inner_ws_smem<GE>(MAX_L));
     else return cudaSuccess;
 }
 
@@ -1371,8 +1372,9 @@ static cudaError_t launch_inner_ws(const pc_ctx *c, dim3 grid, cudaStream_t s, c
                                    int pi, u32 t0) {
     using GE = Geo<LG>;
     if constexpr (LastPhase<GE::LOGC>::type::KK == 16)
-        return launch_ex(c, k_inner_ws<LG>, grid, dim3(2 * GE::ROW_THREADS), inner_ws_smem<GE>(), s, c->tab, src,
-                         srcz, c1, c1z, acc, accz, l, kp, pi, t0);
+        return launch_ex(c, k_inner_ws<LG>, grid, dim3(2 * GE::ROW_THREADS),
+                         inner_ws_smem<GE>((l + c->alpha - 1) / c->alpha), s, c->tab, src, srcz, c1, c1z, acc, accz,
+                         l, kp, pi, t0);
     else
         return cudaErrorInvalidValue;
 }
