@@ -267,7 +267,9 @@ struct Geo {
     // per TPCOL consecutive lanes, CPW columns per warp, warp barriers only
     static constexpr int CPW = 32 / TPCOL;
     static constexpr int COL_LS = R + R / 16;  // padded column stride in shared memory
-    static constexpr int COL_LS4 = R + R / 4;  // column stride of a Pad4Addr line
+    // column stride of a Pad4Addr line (+16 words: a warp's two columns on
+    // opposite bank halves)
+    static constexpr int COL_LS4 = R + R / 4 + 16;
     static_assert(LOGC >= 4 && LOGR >= 4 && LOGR <= 9, "supported 2^8..2^17 (R,C >= 16)");
 };
 
