@@ -51,7 +51,7 @@ L2_BYTES = 126 * 2**20
 # from one ncu capture (--clock-control none, cold cache) of the kernel source
 # whose hash is given; reported only while the kernel sources still hash to
 # that value (otherwise the traffic is null: the counters are stale).
-KERNEL_TRAFFIC = {("rot1_n16", "inner_chacha"): (104.93e6 + 5.13e6, "0000000000000000")}
+KERNEL_TRAFFIC = {("rot1_n16", "inner_chacha"): (104.933376e6 + 6.021632e6, "1890608946a0677e")}
 KERNEL_SOURCES = ("kernels.cu", "ntt.cuh", "chacha.cuh", "modarith.cuh")
 
 

@@ -61,11 +61,12 @@ def test_linear_transform_two_baby_batches(built, oracle):
     _run(oracle, P, C, 4, 18, 2, 3)
 
 
-@pytest.mark.parametrize("l", [23, 5])
-def test_linear_transform_n17_levels(built, oracle, l):
-    """N=2^17, L=40, alpha=5, dnum=8 at sampled levels, n1 = n2 = 3."""
+@pytest.mark.parametrize("l,n1,n2", [(23, 3, 3), (5, 4, 4), (40, 2, 2)])
+def test_linear_transform_n17_levels(built, oracle, l, n1, n2):
+    """N=2^17, L=40, alpha=5, dnum=8 at sampled levels of the sweep: the
+    bench's 4 x 4 shape at a low level, the top level with 2 x 2."""
     P, C = G.contexts(oracle, 17, 40, 5, 31)
-    _run(oracle, P, C, l, 3, 3, 40 + l)
+    _run(oracle, P, C, l, n1, n2, 40 + l)
 
 
 def test_linear_transform_errors(built, oracle):
