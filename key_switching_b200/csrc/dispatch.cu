@@ -48,7 +48,7 @@ PC_NS_END
         default: return cudaErrorInvalidValue;                                  \
     }
 
-cudaError_t prepare_kernels(const pc_ctx *c) { PC_FORWARD(prepare_kernels, c) }
+cudaError_t prepare_kernels(pc_ctx *c) { PC_FORWARD(prepare_kernels, c) }
 
 cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
                        size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s, u32 galois,

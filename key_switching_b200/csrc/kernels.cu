@@ -352,8 +352,9 @@ k_col(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zou
 // 16-byte accesses on distinct bank groups.
 constexpr int YT_LS = 20;
 
-// One CTA of alpha warps per (unit, strip of CPW columns); a column is held
-// by TPCOL consecutive lanes, so every exchange is warp-synchronous.
+// One CTA of alpha warps per item (unit, strip of CPW columns), or per part of
+// an item's targets; a column is held by TPCOL consecutive lanes, so every
+// exchange is warp-synchronous.
 //   mode 0 (ModUp):   unit = digit j; warp k < d runs the inverse column pass
 //                     of limb q_{j alpha + k} (column-major input) times
 //                     N^-1 [Dhat_k^-1]; targets t not in D_j -> out[j][t]
@@ -363,10 +364,11 @@ constexpr int YT_LS = 20;
 // The warps then share the y tiles through shared memory and take the
 // targets round-robin: z_t = sum_k y_k [hat_k]_t (Montgomery constants, one
 // REDC), forward column pass, store (column-major, or row-major for OUT_CM
-// false).  grid (C / CPW, 1, units * Z), block 32 * alpha.
+// false).  1-D grid over the items (strip, unit, z), strip fastest, each
+// item's targets in `split` parts (colconv_split); block 32 * alpha.
 template <int LOGN, int D, bool OUT_CM>
 __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *out, size_t outz, u32 l, u32 unit,
-                                                u32 z, u32 ntarg, const u32 *sy, u32 *xl0, int c, int lt,
+                                                u32 z, u32 tlo, u32 thi, const u32 *sy, u32 *xl0, int c, int lt,
                                                 int col) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
@@ -390,7 +392,7 @@ __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *
     };
     // one target per warp at a time (a short loop body: the kernel is
     // latency-bound and a two-target body overflowed the instruction cache)
-    for (u32 ti = warp; ti < ntarg; ti += nwarps) {
+    for (u32 ti = tlo + warp; ti < thi; ti += nwarps) {
         u32 g0;
         const u32 *conv0;
         u32 *dst0;
@@ -433,7 +435,7 @@ __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *
 
 template <int LOGN, bool OUT_CM>
 __global__ void __launch_bounds__(32 * MAX_ALPHA, COLCONV_MIN_CTAS)
-k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l) {
+k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l, u32 split) {
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
     using PF = typename PL::P0;
@@ -441,12 +443,15 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
     extern __shared__ __align__(16) u32 dyn[];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int c = lane / GE::TPCOL, lt = lane % GE::TPCOL;
-    const int col = blockIdx.x * GE::CPW + c;
+    // item (strip, unit, z) and the part of its targets this CTA converts
+    constexpr u32 STRIPS = GE::C / GE::CPW;
+    const u32 item = blockIdx.x / split, part = blockIdx.x % split;
+    const int col = (int)(item % STRIPS) * GE::CPW + c;
     u32 *sy = dyn;                                          // [alpha][CPW][TPCOL][YT_LS] y tiles
     // one exchange line per warp and column, after the y tiles
     u32 *xl = dyn + T.alpha * GE::CPW * GE::TPCOL * YT_LS + (warp * GE::CPW + c) * GE::COL_LS4;
     const u32 units = mode == 0 ? (l + T.alpha - 1) / T.alpha : 2;
-    const u32 z = blockIdx.z / units, unit = blockIdx.z % units;
+    const u32 z = item / STRIPS / units, unit = item / STRIPS % units;
     const u32 ll = l + T.alpha;
     u32 d, ntarg, gsrc;
     const u32 *s0;
@@ -477,15 +482,16 @@ k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz
                                                             shoup(v[r + 2], sc.x, sc.y, q), shoup(v[r + 3], sc.x, sc.y, q));
     }
     __syncthreads();
+    const u32 tlo = ntarg * part / split, thi = ntarg * (part + 1) / split;
     switch (d) {  // uniform over the CTA
-        case 1: colconv_targets<LOGN, 1, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        case 2: colconv_targets<LOGN, 2, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        case 3: colconv_targets<LOGN, 3, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        case 4: colconv_targets<LOGN, 4, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        case 5: colconv_targets<LOGN, 5, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        case 6: colconv_targets<LOGN, 6, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        case 7: colconv_targets<LOGN, 7, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
-        default: colconv_targets<LOGN, 8, OUT_CM>(T, mode, out, outz, l, unit, z, ntarg, sy, xl, c, lt, col); break;
+        case 1: colconv_targets<LOGN, 1, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        case 2: colconv_targets<LOGN, 2, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        case 3: colconv_targets<LOGN, 3, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        case 4: colconv_targets<LOGN, 4, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        case 5: colconv_targets<LOGN, 5, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        case 6: colconv_targets<LOGN, 6, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        case 7: colconv_targets<LOGN, 7, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
+        default: colconv_targets<LOGN, 8, OUT_CM>(T, mode, out, outz, l, unit, z, tlo, thi, sy, xl, c, lt, col); break;
     }
 }
 
@@ -1284,7 +1290,7 @@ static cudaError_t allow_inner_ws() {
     else return cudaSuccess;
 }
 
-cudaError_t prepare_kernels(const pc_ctx *c) {
+cudaError_t prepare_kernels(pc_ctx *c) {
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         cudaError_t e = allow_smem(k_row<LG, true, false>, row_smem_bytes<GE>(0));
@@ -1305,7 +1311,14 @@ cudaError_t prepare_kernels(const pc_ctx *c) {
         if (e == cudaSuccess) e = allow_smem(k_modup_finish<LG>, row_smem_bytes<GE>(0));
         if (e == cudaSuccess) e = allow_smem(k_colconv<LG, true>, colconv_smem<GE>(c));
         if (e == cudaSuccess) e = allow_smem(k_colconv<LG, false>, colconv_smem<GE>(c));
+        int per_sm = 0, sms = 0;
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device);
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_colconv<LG, true>, 32 * c->alpha,
+                                                              colconv_smem<GE>(c));
         if (e != cudaSuccess) return e;
+        const char *split = getenv("PC_COLCONV_SPLIT");
+        c->colconv_slots = split && split[0] == '0' ? 0u : (u32)(per_sm * sms);
     });
     return cudaSuccess;
 }
@@ -1347,19 +1360,38 @@ cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 f
     return e;
 }
 
+// Work split of the conversion kernel.  A CTA's time is mostly the latency of
+// its dependent column passes, so a call whose items (unit, strip) fill under
+// a quarter of the device's resident CTAs (small rings) splits every item's
+// targets over `split` CTAs, each redoing the short source passes: at most 4
+// parts, at least alpha targets a part (every warp busy).  Larger calls keep
+// whole items: there the extra CTAs of a split held the SMs longer than the
+// shorter tail saved, and delayed the kernels that overlap the conversion.
+static u32 colconv_split(u32 items, u32 slots, u32 ntarg, u32 alpha) {
+    if (!slots || 4 * items > slots) return 1;
+    u32 k = slots / items;
+    if (k > 4) k = 4;
+    while (k > 1 && ntarg / k < alpha) --k;
+    return k;
+}
+
 cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l,
                            u32 Z, bool out_cm, cudaStream_t s) {
     const u32 units = mode == 0 ? (l + c->alpha - 1) / c->alpha : 2;
+    // fewest targets of a unit: l + alpha - d with d <= min(alpha, l) (ModUp), or l (ModDown)
+    const u32 ntarg = mode == 0 ? (l > c->alpha ? l : c->alpha) : l;
     cudaError_t e = cudaSuccess;
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
-        dim3 grid(GE::C / GE::CPW, 1, units * Z);
+        const u32 items = (u32)(GE::C / GE::CPW) * units * Z;
+        const u32 split = colconv_split(items, c->colconv_slots, ntarg, c->alpha);
+        const dim3 grid(items * split);
         if (out_cm)
             e = launch_ex(c, k_colconv<LG, true>, grid, dim3(32 * c->alpha), colconv_smem<GE>(c), s, c->tab, mode,
-                          src, srcz, out, outz, l);
+                          src, srcz, out, outz, l, split);
         else
             e = launch_ex(c, k_colconv<LG, false>, grid, dim3(32 * c->alpha), colconv_smem<GE>(c), s, c->tab, mode,
-                          src, srcz, out, outz, l);
+                          src, srcz, out, outz, l, split);
     });
     return e;
 }

@@ -89,6 +89,9 @@ struct pc_ctx {
     // PC_CHECK_* flags of pc_set_checks: validate inputs on the device
     uint32_t checks;
     uint32_t last_err_word;  // the error word pc_check last found set
+    // CTAs of the conversion kernel resident at once on the device (0: never
+    // split its items by target; PC_COLCONV_SPLIT=0)
+    uint32_t colconv_slots;
     // launch attributes: programmatic dependent launch, L2 persistence of the tables
     int use_pdl;
     void *l2_window_base;
@@ -180,7 +183,9 @@ struct DeviceGuard {
     DeviceGuard(const DeviceGuard &) = delete;
     DeviceGuard &operator=(const DeviceGuard &) = delete;
 };
-cudaError_t prepare_kernels(const pc_ctx *c);
+// Per-degree set-up: shared-memory limits of the kernels and the number of
+// conversion-kernel CTAs resident on the device (colconv_slots)
+cudaError_t prepare_kernels(pc_ctx *c);
 
 // Remember a CUDA error for pc_strerror(PC_E_CUDA); returns PC_E_CUDA.
 int record_cuda_error(cudaError_t e);
