@@ -54,6 +54,7 @@ extern "C" {
 #define PC_E_PRIME (-6)     /* a modulus is not prime, not = 1 mod 2N, or >= 2^31 */
 #define PC_E_WORKSPACE (-7) /* no workspace set, or smaller than pc_workspace_bytes */
 #define PC_E_TOO_BIG (-8)   /* size beyond the static scratch of pc_modup_noalloc */
+#define PC_E_UNSUPPORTED (-9) /* the call needs a library built with the per-CTA timeline */
 
 typedef struct pc_ctx pc_ctx; /* opaque; owns the device constant tables */
 typedef void *pc_stream;      /* a cudaStream_t */
@@ -354,6 +355,33 @@ int pc_microbench(int device, int kind, uint32_t iters, double *ops_per_s);
 #define PC_PROFILE_STAGES 5
 int pc_profile_begin(pc_ctx *ctx, uint32_t max_calls, uint32_t every);
 int pc_profile_end(pc_ctx *ctx, float *ms, uint32_t *calls);
+
+/* Per-CTA timeline of the key-switching kernels, for measurement.  Only a
+ * library built with it (python -m key_switching_b200.build --timeline, which
+ * writes libpc_timeline.so) records it: there every CTA of the kernels below
+ * stores, as it exits, its start and end time (the GPU's global nanosecond
+ * timer) and its SM id into a device array of PC_TL_ROLES x PC_TL_CTAS
+ * records, at [role][CTA index within its grid], so each record holds the
+ * latest launch of that role.  pc_timeline_read synchronises the context's
+ * device, copies the array to host memory `out` (PC_TL_ROLES * PC_TL_CTAS * 3
+ * uint64 words: start ns, end ns, SM) and zeroes it.  Roles: the inverse row
+ * pass of c1 (ModUp), the conversion kernels of ModUp and ModDown, the inner
+ * products of the special-prime and of the ciphertext-prime limbs
+ * (two-group kernel), the ModDown finish, other row passes, the single-group
+ * and rotation inner products.  CTAs beyond PC_TL_CTAS are not recorded.
+ * Returns PC_OK, PC_E_ARG (null or `words` too small), PC_E_UNSUPPORTED
+ * (default build) or PC_E_CUDA. */
+#define PC_TL_ROLES 8
+#define PC_TL_CTAS 4096
+#define PC_TL_ROW_C1 0
+#define PC_TL_CONV_UP 1
+#define PC_TL_INNER_SPECIAL 2
+#define PC_TL_CONV_DOWN 3
+#define PC_TL_INNER_CT 4
+#define PC_TL_MODDOWN_FINISH 5
+#define PC_TL_ROW_OTHER 6
+#define PC_TL_INNER_OTHER 7
+int pc_timeline_read(pc_ctx *ctx, uint64_t *out, size_t words);
 
 #ifdef __cplusplus
 }

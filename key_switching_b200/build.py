@@ -3,8 +3,11 @@
     python -m key_switching_b200.build [--force]
 
 Produces key_switching_b200/libpc.so from key_switching_b200/csrc/*.cu (the
-kernel file once per ring degree, -DPC_LOGN=10..17, all in parallel).  No GPU
-is needed to build (nvcc cross-compiles).
+kernel file once per ring degree, -DPC_LOGN=10..17, all in parallel).  With
+--timeline it builds key_switching_b200/libpc_timeline.so instead: the same
+library compiled with -DPC_TIMELINE, whose kernels record the per-CTA timeline
+that pc_timeline_read returns (loaded by the binding when PC_TIMELINE=1).  No
+GPU is needed to build (nvcc cross-compiles).
 """
 from __future__ import annotations
 
@@ -16,6 +19,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpc.so")
+LIB_TIMELINE = os.path.join(HERE, "libpc_timeline.so")
 ROOT = os.path.dirname(HERE)
 
 NVCC_FLAGS = [
@@ -40,30 +44,32 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(CSRC, "*.inc"))
     deps.append(os.path.join(ROOT, "include", "pc.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, timeline: bool = False) -> str:
     """Compile every csrc/*.cu to an object (in parallel, one nvcc per file)
-    and link them into libpc.so; a no-op when the library is newer than every
-    source."""
-    if not force and not needs_build():
-        return LIB
+    and link them into libpc.so (libpc_timeline.so with timeline=True); a
+    no-op when the library is newer than every source."""
+    lib = LIB_TIMELINE if timeline else LIB
+    if not force and not needs_build(lib):
+        return lib
     from concurrent.futures import ThreadPoolExecutor
-    objdir = os.path.join(HERE, "_build")
+    objdir = os.path.join(HERE, "_build", "timeline" if timeline else "default")
+    extra = ["-DPC_TIMELINE"] if timeline else []
     os.makedirs(objdir, exist_ok=True)
     inc = ["-I", os.path.join(ROOT, "include")]
 
     def compile_one(src, name, defs):
         obj = os.path.join(objdir, name + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, *defs, *inc, "-c", "-o", obj, src]
+        cmd = [nvcc(), *NVCC_FLAGS, *extra, *defs, *inc, "-c", "-o", obj, src]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
@@ -79,14 +85,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
             jobs.append((src, os.path.basename(src)[:-3], []))
     with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
         objs = list(ex.map(lambda j: compile_one(*j), jobs))
-    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB + ".tmp", *objs]
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", lib + ".tmp", *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, timeline="--timeline" in sys.argv))

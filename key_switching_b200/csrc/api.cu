@@ -1059,6 +1059,14 @@ int pc_profile_end(pc_ctx *c, float *ms, uint32_t *calls) {
     return rc;
 }
 
+int pc_timeline_read(pc_ctx *c, uint64_t *out, size_t words) {
+    if (!c || !out || words < (size_t)PC_TL_ROLES * PC_TL_CTAS * 3) return PC_E_ARG;
+    DeviceGuard dg(c->device);
+    const cudaError_t e = pc::timeline_read(c, out);
+    if (e == cudaErrorNotSupported) return PC_E_UNSUPPORTED;
+    return e == cudaSuccess ? PC_OK : cuda_fail(e);
+}
+
 int pc_check(pc_ctx *c) {
     if (!c) return PC_E_ARG;
     DeviceGuard dg(c->device);
@@ -1094,6 +1102,7 @@ const char *pc_strerror(int code) {
         case PC_E_PRIME: return "modulus not prime, not 1 mod 2N, repeated, or >= 2^31";
         case PC_E_WORKSPACE: return "workspace missing or smaller than pc_workspace_bytes";
         case PC_E_TOO_BIG: return "l*N exceeds the static scratch of pc_modup_noalloc (2^21 words)";
+        case PC_E_UNSUPPORTED: return "the library was built without the per-CTA timeline (build --timeline)";
         default: return "unknown status code";
     }
 }

@@ -50,6 +50,8 @@ PC_NS_END
 
 cudaError_t prepare_kernels(pc_ctx *c) { PC_FORWARD(prepare_kernels, c) }
 
+cudaError_t timeline_read(const pc_ctx *c, uint64_t *out) { PC_FORWARD(timeline_read, c, out) }
+
 cudaError_t launch_row(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 first_prime, u32 nlimbs, u32 Z,
                        size_t zin, size_t zout, bool canonical, bool cm_out, cudaStream_t s, u32 galois,
                        const u32 *mul, u32 *xout, const MacIn *mac) {

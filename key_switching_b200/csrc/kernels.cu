@@ -61,6 +61,39 @@ constexpr int COLCONV_MIN_CTAS = PC_COLCONV_MIN_CTAS;
 constexpr int INNER_MIN_CTAS = PC_INNER_MIN_CTAS;
 constexpr int MODDOWN_MIN_CTAS = PC_MODDOWN_MIN_CTAS;
 
+// ------------------------------------------------------- per-CTA timeline
+// Built with -DPC_TIMELINE only: each key-switching kernel stamps its CTA's
+// start and end (%globaltimer, ns) and SM id, as the CTA's thread 0 exits,
+// into g_tl[role][CTA index]; timeline_read copies the array out.
+#ifdef PC_TIMELINE
+namespace {
+__device__ unsigned long long g_tl[PC_TL_ROLES][PC_TL_CTAS][3];
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+struct TlStamp {
+    int role;
+    unsigned long long t0;
+    __device__ explicit TlStamp(int r) : role(r), t0(global_ns()) {}
+    __device__ ~TlStamp() {
+        if (threadIdx.x != 0) return;
+        const unsigned b = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+        if (b >= PC_TL_CTAS) return;
+        unsigned sm;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+        g_tl[role][b][0] = t0;
+        g_tl[role][b][1] = global_ns();
+        g_tl[role][b][2] = sm;
+    }
+};
+#define PC_TL(role) const TlStamp pc_tl_stamp_(role)
+#else
+#define PC_TL(role) ((void)0)
+#endif
+
 // ------------------------------------------------------------------ helpers
 
 // global prime index of local limb t at level l
@@ -245,6 +278,7 @@ template <int LOGN, bool FWD, bool CMOUT, bool MAC = false>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, ROW_MIN_CTAS)
 k_row(Tables T, const u32 *in, u32 *out, u32 first_prime, size_t zin, size_t zout, int canonical, u32 galois,
       const u32 *mul, u32 *xout, MacIn mac) {
+    PC_TL(CMOUT ? PC_TL_ROW_C1 : PC_TL_ROW_OTHER);
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -436,6 +470,7 @@ __device__ __forceinline__ void colconv_targets(const Tables &T, int mode, u32 *
 template <int LOGN, bool OUT_CM>
 __global__ void __launch_bounds__(32 * MAX_ALPHA, COLCONV_MIN_CTAS)
 k_colconv(Tables T, int mode, const u32 *src, size_t srcz, u32 *out, size_t outz, u32 l, u32 split) {
+    PC_TL(mode == 0 ? PC_TL_CONV_UP : PC_TL_CONV_DOWN);
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGR>;
     using PF = typename PL::P0;
@@ -708,6 +743,7 @@ template <int LOGN, bool FUSED, bool REGEN>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, INNER_MIN_CTAS)
 k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz,
         u32 l, KeyPack kp, int pintt, u32 t0) {
+    PC_TL(PC_TL_INNER_OTHER);
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -882,6 +918,7 @@ template <int LOGN>
 __global__ void __launch_bounds__(2 * Geo<LOGN>::ROW_THREADS, PC_INNER_WS_MIN_CTAS)
 k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
            KeyPack kp, int pintt, u32 t0) {
+    PC_TL(t0 > 0 ? PC_TL_INNER_SPECIAL : PC_TL_INNER_CT);
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -1058,6 +1095,7 @@ template <int LOGN, bool REGEN>
 __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, INNER_MIN_CTAS)
 k_inner_rot(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
             KeyPack kp, int pintt, u32 t0, RotPack rp) {
+    PC_TL(PC_TL_INNER_OTHER);
     inner_body<LOGN, true, REGEN, true>(T, src, srcz, c1, c1z, acc, accz, l, kp, pintt, t0,
                                         pick(rp.galois, blockIdx.z), pick(rp.ginv, blockIdx.z));
 }
@@ -1077,6 +1115,7 @@ __global__ void __launch_bounds__(Geo<LOGN>::ROW_THREADS, MODDOWN_MIN_CTAS)
 k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, const u32 *c0,
               size_t c0z, u32 *out0, u32 *out1, size_t outz, u32 l, RotPack rp, const u32 *rx, const u32 *ry,
               MacIn mac) {
+    PC_TL(PC_TL_MODDOWN_FINISH);
     using GE = Geo<LOGN>;
     using PL = Plan<GE::LOGC>;
     using PF = typename PL::P0;
@@ -1288,6 +1327,23 @@ static cudaError_t allow_inner_ws() {
     using GE = Geo<LG>;
     if constexpr (LastPhase<GE::LOGC>::type::KK == 16) return allow_smem(k_inner_ws<LG>, inner_ws_smem<GE>(MAX_L));
     else return cudaSuccess;
+}
+
+cudaError_t timeline_read(const pc_ctx *c, uint64_t *out) {
+    (void)c;
+#ifdef PC_TIMELINE
+    static_assert(sizeof(g_tl) == sizeof(uint64_t) * PC_TL_ROLES * PC_TL_CTAS * 3, "timeline layout");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(out, g_tl, sizeof(g_tl));
+    void *p = nullptr;
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(&p, g_tl);
+    if (e == cudaSuccess) e = cudaMemset(p, 0, sizeof(g_tl));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    return e;
+#else
+    (void)out;
+    return cudaErrorNotSupported;
+#endif
 }
 
 cudaError_t prepare_kernels(pc_ctx *c) {

@@ -186,6 +186,9 @@ struct DeviceGuard {
 // Per-degree set-up: shared-memory limits of the kernels and the number of
 // conversion-kernel CTAs resident on the device (colconv_slots)
 cudaError_t prepare_kernels(pc_ctx *c);
+// copy out and zero the per-CTA timeline of the context's degree
+// (cudaErrorNotSupported unless built with PC_TIMELINE)
+cudaError_t timeline_read(const pc_ctx *c, uint64_t *out);
 
 // Remember a CUDA error for pc_strerror(PC_E_CUDA); returns PC_E_CUDA.
 int record_cuda_error(cudaError_t e);

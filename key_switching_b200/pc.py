@@ -12,11 +12,13 @@ import os
 from typing import Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpc.so")
+# PC_TIMELINE=1 loads the build whose kernels record the per-CTA timeline
+TIMELINE = os.environ.get("PC_TIMELINE") == "1"
+LIB_PATH = os.path.join(_HERE, "libpc_timeline.so" if TIMELINE else "libpc.so")
 
 PC_OK = 0
 ERRORS = {-1: "PC_E_ARG", -2: "PC_E_ALIGN", -3: "PC_E_CUDA", -4: "PC_E_DEVICE",
-          -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE", -8: "PC_E_TOO_BIG"}
+          -6: "PC_E_PRIME", -7: "PC_E_WORKSPACE", -8: "PC_E_TOO_BIG", -9: "PC_E_UNSUPPORTED"}
 CHECK_INPUTS = 1           # pc_set_checks flag
 ERR_INPUT, ERR_KEY = 1, 2  # bits of the device error word
 
@@ -27,8 +29,13 @@ EXPORTS = ("pc_gen_primes", "pc_ctx_create", "pc_ctx_destroy", "pc_psi", "pc_wor
            "pc_strerror", "pc_microbench", "pc_profile_begin", "pc_profile_end", "pc_modup_noalloc",
            "pc_rotate", "pc_rotate_hoisted", "pc_relinearize", "pc_keyswitch_host", "pc_host_workspace_bytes",
            "pc_keyswitch_capture", "pc_graph_launch", "pc_graph_destroy", "pc_capture_begin", "pc_capture_end",
-           "pc_set_checks", "pc_last_error_word", "pc_linear_transform", "pc_linear_transform_workspace_bytes")
+           "pc_set_checks", "pc_last_error_word", "pc_linear_transform", "pc_linear_transform_workspace_bytes",
+           "pc_timeline_read")
 PROFILE_STAGES = ("intt_row_c1", "modup_col", "inner_chacha", "moddown_col", "moddown_finish")
+# roles of the per-CTA timeline (PC_TL_* of pc.h, in order)
+TL_ROLES = ("row_c1", "conv_up", "inner_special", "conv_down", "inner_ct", "moddown_finish", "row_other",
+            "inner_other")
+TL_CTAS = 4096
 
 
 class PCError(RuntimeError):
@@ -55,8 +62,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m key_switching_b200.build` "
-                              "(the library has no CPU fallback)")
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m key_switching_b200.build"
+                              f"{' --timeline' if TIMELINE else ''}` (the library has no CPU fallback)")
         L = ctypes.CDLL(LIB_PATH)
         u32, i32, vp, sz = ctypes.c_uint32, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
         L.pc_gen_primes.argtypes = [u32, u32, u32, ctypes.POINTER(u32)]
@@ -125,6 +132,8 @@ def lib():
         L.pc_profile_begin.restype = i32
         L.pc_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(u32)]
         L.pc_profile_end.restype = i32
+        L.pc_timeline_read.argtypes = [vp, vp, sz]
+        L.pc_timeline_read.restype = i32
         L.pc_modup_noalloc.argtypes = [vp, vp, u32, vp, vp]
         L.pc_modup_noalloc.restype = i32
         _lib = L
@@ -415,3 +424,13 @@ class Context:
         n = ctypes.c_uint32()
         _ok(lib().pc_profile_end(self._h, ms, ctypes.byref(n)), "pc_profile_end")
         return dict(zip(PROFILE_STAGES, [float(v) for v in ms])), int(n.value)
+
+    def timeline_read(self):
+        """Per-CTA timeline (library built with --timeline, PC_TIMELINE=1):
+        uint64 array [len(TL_ROLES)][TL_CTAS][3] of (start ns, end ns, SM) of
+        each role's latest launch (zeros where no CTA ran); the device copy is
+        zeroed."""
+        import numpy as np
+        out = np.zeros((len(TL_ROLES), TL_CTAS, 3), dtype=np.uint64)
+        _ok(lib().pc_timeline_read(self._h, out.ctypes.data, out.size), "pc_timeline_read")
+        return out

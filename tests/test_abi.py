@@ -65,9 +65,11 @@ def test_ctx_create_rejects_bad_params_before_touching_cuda(pc):
 
 def test_strerror_and_null_args(pc):
     lib = pc.lib()
-    for code in (0, -1, -2, -3, -4, -6, -7, -8):
+    for code in (0, -1, -2, -3, -4, -6, -7, -8, -9):
         assert len(pc.strerror(code)) >= 2
+    assert pc.strerror(-9) != pc.strerror(-100)  # -9 is a known code
     assert lib.pc_ntt_fwd(None, None, 0, 1, 1, None) == -1
+    assert lib.pc_timeline_read(None, None, 0) == -1
     assert lib.pc_keyswitch(None, None, None, 1, None, None, None, None) == -1
     assert lib.pc_workspace_bytes(None, 1, 1) == 0
     assert lib.pc_gen_primes(16, 40, 1, (ctypes.c_uint32 * 1)()) == -1
