@@ -1135,17 +1135,19 @@ k_moddown_row(Tables T, const u32 *U, size_t Uz, const u32 *acc, size_t accz, co
     u32 *line = sm + rho * GE::ROW_LS;
     const TwRow tw{stw + rho * GE::C};
     stage_row_tw<GE>(stw, T.rowF + (size_t)i * GE::N + (size_t)row0 * GE::C);
+    // c0 is the caller's input, which no kernel of the call writes: its row
+    // loads before the wait for the inner products and the ModDown conversion
+    u32 ah[2][16], c0v[16];
+    if constexpr (XF == XF_PLAIN) {
+        if (c0) gload<PLAST>(c0v, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
+    }
     pdl_wait();
     pdl_trigger();
     stage_cm_rows<GE>(tiles, U + z * Uz + (size_t)i * GE::N, row0);
     stage_cm_rows<GE>(tiles + GE::C * 8, U + z * Uz + ((size_t)l + i) * GE::N, row0);
-    // both halves' accumulator rows (and c0's row) load while the tiles stage
-    u32 ah[2][16], c0v[16];
+    // both halves' accumulator rows load while the tiles stage
     gload<PLAST>(ah[0], acc + z * accz + (size_t)i * GE::N + rowoff, lt);
     gload<PLAST>(ah[1], acc + z * accz + ((size_t)ll + i) * GE::N + rowoff, lt);
-    if constexpr (XF == XF_PLAIN) {
-        if (c0) gload<PLAST>(c0v, c0 + z * c0z + (size_t)i * GE::N + rowoff, lt);
-    }
     cp_async_wait_all();
     __syncthreads();
     auto half = [&](const int h) {

@@ -236,7 +236,8 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 // the stream has completed and its writes are visible (a no-op when the
 // kernel was launched without the attribute); pdl_trigger() lets the next
 // grid start launching once every CTA of this grid has called it.  Kernels
-// read only constant tables before pdl_wait() and write nothing before it.
+// read only constant tables (and the ModDown finish the caller's c0, which no
+// kernel of a call writes) before pdl_wait() and write nothing before it.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" :::); }
 
