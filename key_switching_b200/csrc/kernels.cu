@@ -60,6 +60,14 @@ constexpr int ROW_MIN_CTAS = PC_ROW_MIN_CTAS;
 constexpr int COLCONV_MIN_CTAS = PC_COLCONV_MIN_CTAS;
 constexpr int INNER_MIN_CTAS = PC_INNER_MIN_CTAS;
 constexpr int MODDOWN_MIN_CTAS = PC_MODDOWN_MIN_CTAS;
+// depth of the two-group inner product's ring of regenerated 'a' buffers and
+// its named-barrier ids (FULL[s], EMPTY[s]; hardware ids go up to 15)
+#ifndef PC_WS_RING
+#define PC_WS_RING 6
+#endif
+constexpr int WS_RING = PC_WS_RING;
+constexpr int WS_FULL = 2, WS_EMPTY = 2 + WS_RING;
+static_assert(WS_RING >= 2 && WS_EMPTY + WS_RING - 1 <= 15, "named barrier ids");
 
 // ------------------------------------------------------- per-CTA timeline
 // Built with -DPC_TIMELINE only: each key-switching kernel stamps its CTA's
@@ -907,13 +915,16 @@ k_inner(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *a
 // ahead with asynchronous copies, runs the forward row passes and
 // multiply-accumulates both halves.  So the ALU-bound cipher and the
 // multiply-bound transforms run in different warps and overlap on the SM.
-// Hand-off: named barriers FULL[s] (ids 2, 3: the producer arrives once
-// digit j's words are in buffer s = j mod 2, the consumer waits) and
-// EMPTY[s] (ids 4, 5: the consumer arrives once it has read buffer s, if
-// digit j + 2 exists; the producer waits before refilling it); id 1 orders the
-// consumer group alone.  Every thread of a group takes the same barrier
-// steps (beta and the own digit are uniform over the CTA), so each barrier
-// phase completes.
+// The 'a' words pass through a ring of WS_RING buffers: the producer runs up to
+// WS_RING digits ahead -- all of them at N=2^16, l=24 -- which it does while
+// the consumer waits for the conversion kernel to finish.
+// Hand-off: named barriers FULL[s] (ids 2 .. WS_RING + 1: the producer
+// arrives once digit j's words are in buffer s = j mod WS_RING, the consumer
+// waits) and EMPTY[s] (ids WS_RING + 2 .. 2 WS_RING + 1: the consumer arrives
+// once it has read buffer s, if digit j + WS_RING exists; the producer waits
+// before refilling it); id 1 orders the consumer group alone.  Every thread
+// of a group takes the same barrier steps (beta and the own digit are uniform
+// over the CTA), so each barrier phase completes.
 template <int LOGN>
 __global__ void __launch_bounds__(2 * Geo<LOGN>::ROW_THREADS, PC_INNER_WS_MIN_CTAS)
 k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32 *acc, size_t accz, u32 l,
@@ -930,8 +941,8 @@ k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32
     u32 *sm = dyn + 2 * GE::NL * GE::C;                      // [NL][ROW_LS] exchange
     u32 *tiles = sm + GE::NL * GE::ROW_LS;                   // [2][C*8] column-pass tiles
     uint4 *bbuf = reinterpret_cast<uint4 *>(tiles + 2 * GE::C * 8);  // [2][4][NT] key 'b' words
-    u32 *abuf = tiles + 2 * GE::C * 8 + 2 * 16 * NT;          // [2][16][NT] regenerated 'a'
-    u32 *spre = abuf + 2 * 16 * NT;                            // [beta][12] first-round words
+    u32 *abuf = tiles + 2 * GE::C * 8 + 2 * 16 * NT;          // [WS_RING][16][NT] regenerated 'a'
+    u32 *spre = abuf + WS_RING * 16 * NT;                      // [beta][12] first-round words
     const bool producer = threadIdx.x >= NT;
     const int tid = producer ? threadIdx.x - NT : threadIdx.x;
     const int rho = tid / GE::TPR, lt = tid % GE::TPR;
@@ -961,9 +972,8 @@ k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32
 #pragma unroll
         for (int i = 0; i < 8; ++i) seed[i] = kp.seed[z][i];
         const u32 base = (u32)(rowoff + PLAST::x_of(lt, 0));
-        for (u32 j = 0; j < beta; ++j) {
-            const int s = j & 1;
-            if (j >= 2) bar_sync(4 + s, 2 * NT);
+        for (u32 j = 0, s = 0; j < beta; ++j, s = s + 1 == WS_RING ? 0 : s + 1) {
+            if (j >= (u32)WS_RING) bar_sync(WS_EMPTY + s, 2 * NT);
             u32 o0[16], o1[16], pre[12];
             const uint4 *pp = reinterpret_cast<const uint4 *>(spre + 12 * j);
 #pragma unroll
@@ -979,7 +989,7 @@ k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32
                 ab[w * NT] = redc(o0[2 * w], mod32(o0[2 * w + 1], q, pk.q1s), q, pk.qn);
                 ab[(8 + w) * NT] = redc(o1[2 * w], mod32(o1[2 * w + 1], q, pk.q1s), q, pk.qn);
             }
-            bar_arrive(2 + s, 2 * NT);
+            bar_arrive(WS_FULL + s, 2 * NT);
         }
         return;
     }
@@ -1033,11 +1043,12 @@ k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32
             const uint4 w4 = bb[c * NT];
             bv[4 * c] = w4.x; bv[4 * c + 1] = w4.y; bv[4 * c + 2] = w4.z; bv[4 * c + 3] = w4.w;
         }
-        bar_sync(2 + (j & 1), 2 * NT);  // digit j's 'a' words are in
-        const u32 *ab = abuf + (j & 1) * 16 * NT + tid;
+        const u32 slot = j % WS_RING;
+        bar_sync(WS_FULL + slot, 2 * NT);  // digit j's 'a' words are in
+        const u32 *ab = abuf + slot * 16 * NT + tid;
 #pragma unroll
         for (int r = 0; r < 16; ++r) av[r] = ab[r * NT];
-        if (j + 2 < beta) bar_arrive(4 + (j & 1), 2 * NT);
+        if (j + WS_RING < beta) bar_arrive(WS_EMPTY + slot, 2 * NT);
         // multiply-accumulate; fold the 64-bit sums every two digits
         const bool fold = (j & 1) && (j + 1 < beta);
 #pragma unroll
@@ -1296,11 +1307,11 @@ static size_t colconv_smem(const pc_ctx *c) {
     return sizeof(u32) * ((size_t)c->alpha * GE::CPW * GE::TPCOL * YT_LS + (size_t)c->alpha * GE::CPW * GE::COL_LS4);
 }
 
-// k_inner_ws: the key 'b' and regenerated 'a' double buffers of its two
-// groups, and the counter-free first-round words of each of the beta digits
+// k_inner_ws: the key 'b' double buffer, the ring of regenerated 'a'
+// buffers, and the counter-free first-round words of each of the beta digits
 template <class GE>
 static constexpr size_t inner_ws_smem(u32 beta) {
-    return row_smem_bytes<GE>(2) + sizeof(u32) * (2 * 2 * 16 * GE::ROW_THREADS + 12 * (size_t)beta);
+    return row_smem_bytes<GE>(2) + sizeof(u32) * ((2 + WS_RING) * 16 * GE::ROW_THREADS + 12 * (size_t)beta);
 }
 
 // k_inner with ROT: the packed source columns, 4 words per thread
