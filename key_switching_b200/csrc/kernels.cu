@@ -66,8 +66,7 @@ constexpr int MODDOWN_MIN_CTAS = PC_MODDOWN_MIN_CTAS;
 #define PC_WS_RING 6
 #endif
 constexpr int WS_RING = PC_WS_RING;
-constexpr int WS_FULL = 2, WS_EMPTY = 2 + WS_RING;
-static_assert(WS_RING >= 2 && WS_EMPTY + WS_RING - 1 <= 15, "named barrier ids");
+static_assert(WS_RING >= 2 && 2 * WS_RING + 1 <= 15, "named barrier ids 2 .. 2 WS_RING + 1");
 
 // ------------------------------------------------------- per-CTA timeline
 // Built with -DPC_TIMELINE only: each key-switching kernel stamps its CTA's
@@ -943,6 +942,7 @@ k_inner_ws(Tables T, const u32 *src, size_t srcz, const u32 *c1, size_t c1z, u32
     uint4 *bbuf = reinterpret_cast<uint4 *>(tiles + 2 * GE::C * 8);  // [2][4][NT] key 'b' words
     u32 *abuf = tiles + 2 * GE::C * 8 + 2 * 16 * NT;          // [WS_RING][16][NT] regenerated 'a'
     u32 *spre = abuf + WS_RING * 16 * NT;                      // [beta][12] first-round words
+    constexpr int WS_FULL = 2, WS_EMPTY = 2 + WS_RING;  // FULL[s], EMPTY[s] barrier ids
     const bool producer = threadIdx.x >= NT;
     const int tid = producer ? threadIdx.x - NT : threadIdx.x;
     const int rho = tid / GE::TPR, lt = tid % GE::TPR;
