@@ -40,12 +40,15 @@ namespace pc {
 // Minimum resident CTAs per SM given to __launch_bounds__.  Without one,
 // ptxas fits the kernels into 32 registers (full occupancy); these
 // latency-bound kernels run faster with the registers they naturally use
-// (48-105), which keep more independent loads and butterflies in flight.
+// (48-128), which keep more independent loads and butterflies in flight.
+// The conversion kernel's bound is for its largest block (8 warps): 2 CTAs
+// caps it at 128 registers, so that 3 CTAs of 5 warps (alpha = 5, the
+// N=2^17 basis) fit an SM -- unbounded, its N=2^17 build took 146 and 2 fit.
 #ifndef PC_ROW_MIN_CTAS
 #define PC_ROW_MIN_CTAS 8
 #endif
 #ifndef PC_COLCONV_MIN_CTAS
-#define PC_COLCONV_MIN_CTAS 1
+#define PC_COLCONV_MIN_CTAS 2
 #endif
 #ifndef PC_INNER_MIN_CTAS
 #define PC_INNER_MIN_CTAS 4
