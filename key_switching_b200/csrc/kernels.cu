@@ -1437,9 +1437,13 @@ cudaError_t launch_col(const pc_ctx *c, bool fwd, const u32 *in, u32 *out, u32 f
 // a quarter of the device's resident CTAs (small rings) splits every item's
 // targets over `split` CTAs, each redoing the short source passes: at most 4
 // parts, at least alpha targets a part (every warp busy).  Larger calls keep
-// whole items: there the extra CTAs of a split held the SMs longer than the
-// shorter tail saved, and delayed the kernels that overlap the conversion.
-static u32 colconv_split(u32 items, u32 slots, u32 ntarg, u32 alpha) {
+// whole items (the extra CTAs of a split held the SMs longer than the shorter
+// tail saved, and delayed the kernels that overlap the ModUp conversion),
+// except the ModDown conversion when its items fill between one and two waves
+// (N=2^17: 512 on 444): it runs after the inner products, and the partial
+// second wave of whole items would run alone, so it takes halves.
+static u32 colconv_split(int mode, u32 items, u32 slots, u32 ntarg, u32 alpha) {
+    if (mode == 1 && slots && items > slots && items < 2 * slots && ntarg / 2 >= alpha) return 2;
     if (!slots || 4 * items > slots) return 1;
     u32 k = slots / items;
     if (k > 4) k = 4;
@@ -1456,7 +1460,7 @@ cudaError_t launch_colconv(const pc_ctx *c, int mode, const u32 *src, size_t src
     PC_DISPATCH(c->logN, {
         using GE = Geo<LG>;
         const u32 items = (u32)(GE::C / GE::CPW) * units * Z;
-        const u32 split = colconv_split(items, c->colconv_slots, ntarg, c->alpha);
+        const u32 split = colconv_split(mode, items, c->colconv_slots, ntarg, c->alpha);
         const dim3 grid(items * split);
         if (out_cm)
             e = launch_ex(c, k_colconv<LG, true>, grid, dim3(32 * c->alpha), colconv_smem<GE>(c), s, c->tab, mode,
